@@ -1,0 +1,417 @@
+"""Benchmark of the Atom W4A4 hot path on B200.
+
+One step = the online path of one quantized linear layer over one batch:
+atom_reorder_quant of the fp16 activations (reorder + INT4/INT8 quantize) then
+atom_w4a4_gemm against weights quantized once beforehand (the weights are
+quantized offline in the method, so their quantization is outside the step).
+
+Workload: the Llama-70B-shaped MLP up-projection, A fp16 [8192, 8192]
+(Student-t(4), 128 outlier channels x30), W fp16 [28672, 8192] (N(0, 0.01)),
+seeded synthetic inputs (w4a4_mixed_precision_b200.inputs).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl atom|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own batch against
+its own replica of the quantized weights: there is no data exchange on the
+path, so the scaling is weak and `value` sums the ranks' work over the slowest
+rank's time. `--impl reference` times the CPU oracle (test infrastructure) on
+the host cores on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD_INDEX = 4
+METRIC = "W4A4 GEMM TOPS and % int tensor peak; quantize GB/s and % HBM (1 B200)"
+INT8_OVER_BF16 = 2.0     # nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 P)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "w4a4_mixed_precision_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != _kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:                                   # noqa: BLE001 (no NVML: no clocks)
+            self._h = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                bits = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:                               # noqa: BLE001
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._h is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+
+def cpu_oracle_run(w, A, W, idx, budget_s: float, min_rows: int = 8):
+    """Times the CPU oracle on a growing row sample of the workload until the
+    sample takes at least `budget_s`; returns (ops_per_s, rows, seconds, cores)."""
+    from oracle import c_oracle
+    cores = len(os.sched_getaffinity(0))
+    c_oracle.set_threads(cores)
+    qw = c_oracle.quantize(W, idx)                      # offline weights, not timed
+    rows = min_rows
+    while True:
+        t0 = time.perf_counter()
+        qa = c_oracle.quantize(np.ascontiguousarray(A[:rows]), idx)
+        c_oracle.gemm(*qa, *qw, w.K)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or rows >= w.M:
+            break
+        rows = min(w.M, max(rows * 2, int(rows * budget_s / max(dt, 1e-3) * 1.1)))
+    return 2.0 * rows * w.N * w.K / dt, rows, dt, cores
+
+
+# ----------------------------------------------------------------------------- main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["atom", "reference"], default="atom")
+    ap.add_argument("--workload", type=int, default=WORKLOAD_INDEX)
+    ap.add_argument("--cpu-budget", type=float, default=10.0,
+                    help="seconds of CPU oracle work for the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from w4a4_mixed_precision_b200 import inputs
+    w = inputs.workload(args.workload)
+    workload_cfg = {"workload": f"{w.name} M={w.M} N={w.N} K={w.K}", "M": w.M, "N": w.N, "K": w.K,
+                    "group": 128, "n_outlier": 128, "activations": w.describe(),
+                    "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU",
+                    "l2": "inputs larger than L2 (A fp16 134 MB, packed W 121 MB) and every "
+                          "step writes 470 MB of Y, which evicts L2 between steps"}
+
+    if args.impl == "reference":
+        return run_reference(args, w, workload_cfg, rank)
+
+    import torch
+    import torch.distributed as dist
+    from w4a4_mixed_precision_b200 import atom
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    A_h = inputs.activations(args.workload)
+    W_h = inputs.weights(args.workload)
+    idx_h = inputs.outlier_channels(args.workload)
+
+    A = torch.from_numpy(A_h.view(np.uint16)).to(dev).view(torch.float16)
+    idx = torch.from_numpy(idx_h).to(dev)
+    qw = atom.atom_quant_weights(torch.from_numpy(W_h.view(np.uint16)).to(dev).view(torch.float16),
+                                 idx)
+    qa = atom.empty_quantized(w.M, w.K, dev)
+    y = torch.empty((w.M, w.N), dtype=torch.float16, device=dev)
+    torch.cuda.synchronize()
+    atom.atom_device_status(clear=True)
+
+    stream = torch.cuda.current_stream()
+    n_steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_steps)]
+
+    def step(i=None):
+        if i is not None:
+            ev[i][0].record(stream)
+        atom.atom_reorder_quant(A, idx, out=qa, stream=stream)
+        if i is not None:
+            ev[i][1].record(stream)
+        atom.atom_w4a4_gemm(qa, qw, w.K, y=y, stream=stream)
+        if i is not None:
+            ev[i][2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t_start.record(stream)
+        for i in range(n_steps):
+            step(i)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    status = atom.atom_device_status(clear=True)
+    if status != 0:
+        raise RuntimeError(f"device status {atom.STATUS.get(status, status)} during the timed run")
+
+    elapsed_ms = t_start.elapsed_time(t_end)
+    quant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n_steps)]
+    gemm_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(n_steps)]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # -------- end-to-end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        A_pin = torch.from_numpy(A_h.view(np.uint16)).view(torch.float16).pin_memory()
+        y_pin = torch.empty((w.M, w.N), dtype=torch.float16).pin_memory()
+        a_dev = torch.empty_like(A)
+        e2e_steps = max(3, min(20, n_steps // 10))
+
+        def e2e_step():
+            a_dev.copy_(A_pin, non_blocking=True)
+            atom.atom_reorder_quant(a_dev, idx, out=qa, stream=stream)
+            atom.atom_w4a4_gemm(qa, qw, w.K, y=y, stream=stream)
+            y_pin.copy_(y, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / e2e_steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": round(2.0 * w.M * w.N * w.K * world / (e2e_ms * 1e-3) / 1e12, 2),
+               "unit": "TOPS", "h2d_bytes_per_step": A_h.nbytes,
+               "d2h_bytes_per_step": w.M * w.N * 2, "ms_per_step": round(e2e_ms, 4),
+               "steps": e2e_steps}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_kind = _peaks()
+    ops = 2.0 * w.M * w.N * w.K
+    ms_per_step = elapsed_ms / n_steps
+    value = ops * world / (ms_per_step * 1e-3) / 1e12
+    gemm_avg = statistics.mean(gemm_ms)
+    quant_avg = statistics.mean(quant_ms)
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    gemm_tops = ops / (gemm_avg * 1e-3) / 1e12
+    Kd = w.K - 128
+    quant_bytes = w.M * (2 * w.K + Kd // 2 + 128 + 4 * (w.K // 128))
+    quant_gbs = quant_bytes / (quant_avg * 1e-3) / 1e9
+    gemm_bytes = (w.M + w.N) * (Kd // 2 + 128 + 4 * (w.K // 128)) + w.M * w.N * 2
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": n_steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic (seeded; see w4a4_mixed_precision_b200/inputs.py)",
+        "config": workload_cfg,
+        "gemm_tops": round(gemm_tops, 2),
+        "gemm_frac_int8_peak": round(gemm_tops / int8_peak, 4),
+        "quant_gbs": round(quant_gbs, 1),
+        "quant_frac_hbm": round(quant_gbs / peaks["hbm_gbs"], 4),
+        "kernel_ms": {"reorder_quant": round(quant_avg, 4), "w4a4_gemm": round(gemm_avg, 4)},
+        "roofline": {
+            "kernel": "w4a4_gemm_kernel",
+            "bound": "tensor",
+            "achieved": round(gemm_tops, 2),
+            "peak": round(int8_peak, 1),
+            "unit": "TOPS",
+            "frac": round(gemm_tops / int8_peak, 4),
+            "traffic": _profiled_traffic("w4a4_gemm_kernel"),
+            "algorithmic_bytes": gemm_bytes,
+            "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
+                           f"{INT8_OVER_BF16} (nominal int8:bf16 ratio)",
+        },
+        "roofline_quant": {
+            "kernel": "reorder_quant_kernel",
+            "bound": "hbm",
+            "achieved": round(quant_gbs, 1),
+            "peak": peaks["hbm_gbs"],
+            "unit": "GB/s",
+            "frac": round(quant_gbs / peaks["hbm_gbs"], 4),
+            "traffic": _profiled_traffic("reorder_quant_kernel"),
+            "algorithmic_bytes": quant_bytes,
+            "peak_source": f"{peak_kind} HBM copy",
+        },
+        "clocks": clocks.summary(),
+        "gpu_launches": 2 * n_steps,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        ops_s, rows, dt, cores = cpu_oracle_run(w, A_h, W_h, idx_h, args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(ops_s / 1e12, 6), "unit": "TOPS", "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"first {rows} of {w.M} activation rows x all {w.N} "
+                                          f"weight rows (quantize + GEMM, {dt:.1f} s; weights "
+                                          f"quantized beforehand, untimed)"}
+    print(json.dumps(line), flush=True)
+
+
+def run_reference(args, w, workload_cfg, rank):
+    """The CPU oracle as the reference arm: one bounded row sample per step."""
+    if rank != 0:
+        return
+    from w4a4_mixed_precision_b200 import inputs
+    from oracle import c_oracle
+    cores = len(os.sched_getaffinity(0))
+    c_oracle.set_threads(cores)
+    A = inputs.activations(args.workload)
+    W = inputs.weights(args.workload)
+    idx = inputs.outlier_channels(args.workload)
+    qw = c_oracle.quantize(W, idx)
+    # size the per-step sample so that warmup + steps stay within a few minutes
+    t0 = time.perf_counter()
+    probe = 4
+    qa = c_oracle.quantize(np.ascontiguousarray(A[:probe]), idx)
+    c_oracle.gemm(*qa, *qw, w.K)
+    per_row = (time.perf_counter() - t0) / probe
+    total_steps = args.steps + max(3, args.warmup)
+    rows = int(max(1, min(w.M, 120.0 / total_steps / max(per_row, 1e-6))))
+    times = []
+    for i in range(total_steps):
+        t0 = time.perf_counter()
+        qa = c_oracle.quantize(np.ascontiguousarray(A[:rows]), idx)
+        c_oracle.gemm(*qa, *qw, w.K)
+        dt = time.perf_counter() - t0
+        if i >= max(3, args.warmup):
+            times.append(dt)
+    ms = statistics.mean(times) * 1e3
+    value = 2.0 * rows * w.N * w.K / (ms * 1e-3) / 1e12
+    sample = (f"first {rows} of {w.M} activation rows x all {w.N} weight rows per step "
+              f"(quantize + GEMM; weights quantized once beforehand)")
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded; see w4a4_mixed_precision_b200/inputs.py)",
+        "config": workload_cfg, "impl": "reference",
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

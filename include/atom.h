@@ -1,0 +1,170 @@
+/*
+ * atom.h -- C ABI of the Atom W4A4 mixed-precision hot path on B200 (sm_100a).
+ *
+ * The method: "Atom: Low-bit Quantization for Efficient and Accurate LLM
+ * Serving" (arXiv abstract: 4-bit weights and 4-bit activations with a
+ * mixed-precision, fine-grained quantization process; paper summary: per-group
+ * scales and separate higher-precision outlier channels, a dedicated outlier
+ * path for activations) and the quantization record "Atom (mixed-precision
+ * block-outlier low-bit quantization for serving)" (fields "Weight group size":
+ * 128; "notes": every contiguous run of 128 elements is one independently
+ * quantized group, and the high-precision channel size is 128).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - G = K/128 groups per row. Groups 0..G-2 are INT4 groups over the K-128
+ *    non-outlier channels; group G-1 is the INT8 group over the 128 outlier
+ *    channels.
+ *  - Reorder: reordered position j < K-128 holds the j-th non-outlier channel
+ *    in ascending channel order; positions K-128..K-1 hold outlier_idx[0..127]
+ *    in list order.
+ *  - Codes are symmetric, round half to even: q = rint(fp32(x * inv)) with
+ *    scale = amax/qmax and inv = qmax/amax (fp32 divisions; qmax 7 or 127;
+ *    amax = 0 gives scale 0 and zero codes).
+ *  - q4 layout: uint8 [rows][(K-128)/2], row-contiguous; byte i holds elements
+ *    2i (low nibble) and 2i+1 (high nibble) as 4-bit two's complement.
+ *    q8 layout: int8 [rows][128]. scales: float32 [G][rows] (group-major).
+ *  - Every pointer is device memory owned by the caller; the library never
+ *    allocates, frees or synchronises. Work is enqueued on `stream`.
+ *  - Errors a host check can see (null pointers, sizes, alignment, unsupported
+ *    parameters) are returned before anything is launched. Errors only the
+ *    device can see (a repeated or out-of-range outlier index, a bounded wait
+ *    that ran out) are recorded in a device status word that
+ *    atom_device_status() reads.
+ *  - Inputs must be finite.
+ *
+ * Thread safety: the entry points keep no host state except a per-device
+ * cache of the SM count; concurrent calls on different streams are safe.
+ */
+#ifndef ATOM_B200_H
+#define ATOM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATOM_API __attribute__((visibility("default")))
+#else
+#define ATOM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st *atom_stream_t;
+
+typedef enum atom_status {
+    ATOM_OK = 0,
+    ATOM_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad outlier list */
+    ATOM_ERR_SHAPE = 2,        /* K not a multiple of 128, K < 256, N not a multiple of 8, ... */
+    ATOM_ERR_ALIGN = 3,        /* pointer or leading dimension not 16-byte aligned */
+    ATOM_ERR_UNSUPPORTED = 4,  /* group != 128 or n_outlier != 128, or no sm_100 device */
+    ATOM_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+    ATOM_ERR_TIMEOUT = 6       /* a device-side bounded wait gave up (device status only) */
+} atom_status_t;
+
+/*
+ * atom_reorder_quant -- fused activation quantizer (the online path).
+ *
+ * Source: Atom paper summary ("activations get a dedicated outlier path"),
+ * record field "Activation scheme" (outlier channels at higher precision, dense
+ * bulk 4-bit) and "notes" (group 128, 128 high-precision channels).
+ *
+ *   x            fp16 [M][ld_x] device, row-major; only the first K columns are read.
+ *   M            rows (tokens), M >= 0 (M == 0 is a no-op).
+ *   K            channels; K % 128 == 0, 256 <= K <= 32768.
+ *   ld_x         row stride of x in elements, ld_x >= K, ld_x % 8 == 0.
+ *   outlier_idx  int32 [n_outlier] device: distinct channels in [0, K); the list
+ *                order is the order of the outlier codes in q8.
+ *   n_outlier    must be 128.      group: must be 128.
+ *   q4           uint8 [M][(K-128)/2] device (output).
+ *   q8           int8  [M][128]       device (output).
+ *   scales       float [K/128][M]     device (output).
+ * Pointers x, q4, q8 must be 16-byte aligned; scales and outlier_idx 4-byte.
+ * A repeated or out-of-range outlier index makes the kernel write nothing and
+ * sets the device status to ATOM_ERR_INVALID_ARG.
+ */
+ATOM_API atom_status_t atom_reorder_quant(const void *x, int64_t M, int64_t K, int64_t ld_x,
+                                 const int32_t *outlier_idx, int32_t n_outlier, int32_t group,
+                                 uint8_t *q4, int8_t *q8, float *scales, atom_stream_t stream);
+
+/*
+ * atom_quant_weights -- the offline weight quantizer.
+ *
+ * Source: Atom paper summary ("weights are grouped into small blocks ... with
+ * per-group scales"; the outlier channels get the same permutation as the
+ * activations so that the contraction pairs matching channels).
+ *
+ * Same arguments and layouts as atom_reorder_quant with W fp16 [N][ld_w] in
+ * place of x: qw4 [N][(K-128)/2], qw8 [N][128], sw [K/128][N]. The weight
+ * layout is exactly the activation layout, so the oracle compares it directly.
+ */
+ATOM_API atom_status_t atom_quant_weights(const void *w, int64_t N, int64_t K, int64_t ld_w,
+                                 const int32_t *outlier_idx, int32_t n_outlier, int32_t group,
+                                 uint8_t *qw4, int8_t *qw8, float *sw, atom_stream_t stream);
+
+/*
+ * atom_w4a4_gemm -- mixed-precision group-scaled integer GEMM.
+ *
+ * Source: Atom abstract (low-bit integer operators for the 4-bit
+ * weight-activation product) and record field "Kernels" (purpose-built low-bit
+ * kernels). Computes, for every m < M and n < N,
+ *
+ *   Y[m][n] = fp16( sum_g sa[g][m] * sw[g][n] * P[g][m][n] ),
+ *   P[g][m][n] = sum over the 128 reordered positions k of group g of qa[m][k]*qw[n][k],
+ *
+ * with exact int32 partials on the tensor cores and an fp32 accumulation of the
+ * dequantized partials (summation order unspecified).
+ *
+ *   qa4, qa8, sa   activation codes/scales as written by atom_reorder_quant (M rows).
+ *   qw4, qw8, sw   weight codes/scales as written by atom_quant_weights (N rows).
+ *   y              fp16 [M][N] device (output), row-major.
+ *   M >= 0, N >= 8 with N % 8 == 0, K as above; n_outlier == group == 128.
+ *   workspace      reserved; may be NULL when workspace_bytes is 0.
+ *                  atom_gemm_workspace_bytes() returns the size needed.
+ * Pointers qa4, qw4, qa8, qw8, y must be 16-byte aligned; sa, sw 4-byte.
+ */
+ATOM_API atom_status_t atom_w4a4_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa,
+                             const uint8_t *qw4, const int8_t *qw8, const float *sw,
+                             void *y, int64_t M, int64_t N, int64_t K,
+                             int32_t n_outlier, int32_t group,
+                             void *workspace, size_t workspace_bytes, atom_stream_t stream);
+
+/*
+ * atom_w4a4_gemm_partials -- debug twin of atom_w4a4_gemm that also writes the
+ * per-group integer partial sums P (same definition as above).
+ *
+ *   partials  int32 [K/128][M][N] device (output).
+ *   y         fp16 [M][N] device (output) or NULL to skip it.
+ * Runs the same tensor-core mainloop as atom_w4a4_gemm. Meant for small shapes:
+ * the partials tensor is G times the size of Y.
+ */
+ATOM_API atom_status_t atom_w4a4_gemm_partials(const uint8_t *qa4, const int8_t *qa8, const float *sa,
+                                      const uint8_t *qw4, const int8_t *qw8, const float *sw,
+                                      int32_t *partials, void *y,
+                                      int64_t M, int64_t N, int64_t K,
+                                      int32_t n_outlier, int32_t group, atom_stream_t stream);
+
+/* Bytes of workspace atom_w4a4_gemm needs for this shape (currently always 0). */
+ATOM_API size_t atom_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * atom_device_status -- first device-detected error since the last clear on the
+ * current device (ATOM_OK if none). Synchronises the current device. With
+ * clear != 0 the status is reset to ATOM_OK afterwards.
+ */
+ATOM_API atom_status_t atom_device_status(int clear);
+
+/* Static, human-readable name of a status code. */
+ATOM_API const char *atom_status_string(atom_status_t status);
+
+/* Library ABI version: major*10000 + minor*100 + patch. */
+ATOM_API int atom_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATOM_B200_H */

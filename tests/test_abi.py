@@ -1,0 +1,119 @@
+"""The C ABI library without a GPU: it loads, exports every entry point that
+include/atom.h declares, and rejects bad arguments on the host before any CUDA
+call (so these checks run on a machine with no GPU at all)."""
+import ctypes as ct
+import os
+import re
+
+import pytest
+
+from w4a4_mixed_precision_b200 import atom
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "atom.h")
+
+OK, INVALID, SHAPE, ALIGN, UNSUPPORTED = 0, 1, 2, 3, 4
+
+# fake, never-dereferenced device addresses: aligned and misaligned
+A16 = 0x10000
+MIS = 0x10001
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(atom_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w4a4_mixed_precision_b200 import build
+    build.build()
+    return atom.lib()
+
+
+def test_header_declares_the_hot_path_entry_points():
+    names = declared_functions()
+    for required in ("atom_reorder_quant", "atom_quant_weights", "atom_w4a4_gemm",
+                     "atom_w4a4_gemm_partials"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) <= set(atom.SIGNATURES)
+
+
+def test_status_strings_and_version(lib):
+    for code, name in atom.STATUS.items():
+        assert atom.atom_status_string(code) == name
+    assert atom.atom_status_string(99) == "ATOM_ERR_UNKNOWN"
+    assert atom.atom_version() >= 100
+    assert atom.atom_gemm_workspace_bytes(8192, 28672, 8192) == 0
+
+
+def quant(lib, x=A16, M=4, K=512, ld=512, idx=A16, n_out=128, group=128, q4=A16, q8=A16,
+          sc=A16, fn="atom_reorder_quant"):
+    return getattr(lib, fn)(x, M, K, ld, idx, n_out, group, q4, q8, sc, None)
+
+
+@pytest.mark.parametrize("fn", ["atom_reorder_quant", "atom_quant_weights"])
+@pytest.mark.parametrize("kw,expect", [
+    (dict(K=500, ld=504), SHAPE),          # K not a multiple of 128
+    (dict(K=128, ld=128), SHAPE),          # K < 256 (needs one INT4 group + the outlier group)
+    (dict(K=65536, ld=65536), SHAPE),      # K above the staged-permutation limit
+    (dict(ld=508), SHAPE),                 # ld < K
+    (dict(ld=516), SHAPE),                 # ld not a multiple of 8 (16-byte rows)
+    (dict(group=64), UNSUPPORTED),
+    (dict(n_out=64), UNSUPPORTED),
+    (dict(M=-1), INVALID),
+    (dict(x=0), INVALID),
+    (dict(idx=0), INVALID),
+    (dict(q4=0), INVALID),
+    (dict(sc=0), INVALID),
+    (dict(x=MIS), ALIGN),
+    (dict(q8=A16 + 8), ALIGN),
+    (dict(sc=A16 + 2), ALIGN),
+    (dict(M=0), OK),                       # empty input: nothing to do, nothing launched
+])
+def test_quantizer_host_validation(lib, fn, kw, expect):
+    assert quant(lib, fn=fn, **kw) == expect
+
+
+def gemm(lib, qa4=A16, qa8=A16, sa=A16, qw4=A16, qw8=A16, sw=A16, y=A16, M=16, N=256, K=512,
+         n_out=128, group=128):
+    return lib.atom_w4a4_gemm(qa4, qa8, sa, qw4, qw8, sw, y, M, N, K, n_out, group, None, 0, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(K=384 + 64), SHAPE),
+    (dict(N=260), SHAPE),                  # N must be a multiple of 8
+    (dict(N=0), SHAPE),
+    (dict(M=-3), INVALID),
+    (dict(y=0), INVALID),
+    (dict(sw=0), INVALID),
+    (dict(qa4=MIS), ALIGN),
+    (dict(y=A16 + 4), ALIGN),
+    (dict(group=256), UNSUPPORTED),
+    (dict(M=0), OK),
+])
+def test_gemm_host_validation(lib, kw, expect):
+    assert gemm(lib, **kw) == expect
+
+
+def test_partials_host_validation(lib):
+    f = lib.atom_w4a4_gemm_partials
+    args = [A16] * 6
+    assert f(*args, 0, A16, 16, 256, 512, 128, 128, None) == INVALID      # no partials buffer
+    assert f(*args, A16 + 4, None, 16, 256, 512, 128, 128, None) == ALIGN
+    assert f(*args, A16, None, 16, 250, 512, 128, 128, None) == SHAPE
+    assert f(*args, A16, None, 0, 256, 512, 128, 128, None) == OK
+
+
+def test_python_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros((4, 256), dtype=torch.float16)
+    idx = torch.arange(128, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        atom.atom_reorder_quant(x, idx)

@@ -1,0 +1,201 @@
+"""Python binding of the C ABI in include/atom.h (argument marshalling only).
+
+Every function here forwards to `libatom_b200.so`: the tensors' device
+pointers, sizes and the current CUDA stream go in, a status code comes back,
+and any status other than ATOM_OK raises AtomError. There is no fallback: if
+the library is missing or the device is not an sm_100 part, the calls fail.
+
+Layouts (see include/atom.h): for R rows of K channels with G = K/128,
+  q4     uint8  [R, (K-128)/2]   two INT4 codes per byte, element 2i low nibble
+  q8     int8   [R, 128]         INT8 codes of the outlier channels, list order
+  scales float32 [G, R]          group-major scales (last row = outlier group)
+"""
+from __future__ import annotations
+
+import ctypes as ct
+import os
+from typing import NamedTuple, Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libatom_b200.so")
+
+STATUS = {
+    0: "ATOM_OK",
+    1: "ATOM_ERR_INVALID_ARG",
+    2: "ATOM_ERR_SHAPE",
+    3: "ATOM_ERR_ALIGN",
+    4: "ATOM_ERR_UNSUPPORTED",
+    5: "ATOM_ERR_CUDA",
+    6: "ATOM_ERR_TIMEOUT",
+}
+
+N_OUTLIER = 128
+GROUP = 128
+
+#: every entry point include/atom.h declares, with its argument types
+SIGNATURES = {
+    "atom_reorder_quant": ([ct.c_void_p, ct.c_int64, ct.c_int64, ct.c_int64, ct.c_void_p,
+                            ct.c_int32, ct.c_int32, ct.c_void_p, ct.c_void_p, ct.c_void_p,
+                            ct.c_void_p], ct.c_int),
+    "atom_quant_weights": ([ct.c_void_p, ct.c_int64, ct.c_int64, ct.c_int64, ct.c_void_p,
+                            ct.c_int32, ct.c_int32, ct.c_void_p, ct.c_void_p, ct.c_void_p,
+                            ct.c_void_p], ct.c_int),
+    "atom_w4a4_gemm": ([ct.c_void_p] * 7 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_int32,
+                                            ct.c_int32, ct.c_void_p, ct.c_size_t, ct.c_void_p],
+                       ct.c_int),
+    "atom_w4a4_gemm_partials": ([ct.c_void_p] * 8 + [ct.c_int64, ct.c_int64, ct.c_int64,
+                                                     ct.c_int32, ct.c_int32, ct.c_void_p],
+                                ct.c_int),
+    "atom_gemm_workspace_bytes": ([ct.c_int64, ct.c_int64, ct.c_int64], ct.c_size_t),
+    "atom_device_status": ([ct.c_int], ct.c_int),
+    "atom_status_string": ([ct.c_int], ct.c_char_p),
+    "atom_version": ([], ct.c_int),
+}
+
+
+class AtomError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib: Optional[ct.CDLL] = None
+
+
+def lib() -> ct.CDLL:
+    """Load libatom_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m w4a4_mixed_precision_b200.build`")
+        handle = ct.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            f = getattr(handle, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = handle
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise AtomError(fn, status)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+class Quantized(NamedTuple):
+    """One quantized operand: INT4 codes, INT8 outlier codes, group-major scales."""
+    q4: torch.Tensor
+    q8: torch.Tensor
+    scales: torch.Tensor
+
+    @property
+    def rows(self) -> int:
+        return self.q4.shape[0]
+
+
+def empty_quantized(rows: int, K: int, device) -> Quantized:
+    return Quantized(torch.empty((rows, (K - N_OUTLIER) // 2), dtype=torch.uint8, device=device),
+                     torch.empty((rows, N_OUTLIER), dtype=torch.int8, device=device),
+                     torch.empty((K // GROUP, rows), dtype=torch.float32, device=device))
+
+
+def _quant(fn: str, x: torch.Tensor, outlier_idx: torch.Tensor, out: Optional[Quantized], stream):
+    if x.dim() != 2:
+        raise ValueError("input must be 2-D [rows, K]")
+    rows, K = x.shape
+    if x.stride(1) != 1:
+        raise ValueError("input rows must be contiguous")
+    if out is None:
+        out = empty_quantized(rows, K, x.device)
+    if not x.is_cuda or x.dtype != torch.float16:
+        raise ValueError("input must be a CUDA float16 tensor")
+    st = getattr(lib(), fn)(x.data_ptr(), rows, K, x.stride(0),
+                            _dev(outlier_idx, torch.int32, "outlier_idx"), outlier_idx.numel(),
+                            GROUP, _dev(out.q4, torch.uint8, "q4"), _dev(out.q8, torch.int8, "q8"),
+                            _dev(out.scales, torch.float32, "scales"), _stream(stream))
+    _check(fn, st)
+    return out
+
+
+def atom_reorder_quant(x: torch.Tensor, outlier_idx: torch.Tensor,
+                       out: Optional[Quantized] = None, stream=None) -> Quantized:
+    """Fused outlier reorder + INT4/INT8 quantization of fp16 activations [M, K]."""
+    return _quant("atom_reorder_quant", x, outlier_idx, out, stream)
+
+
+def atom_quant_weights(w: torch.Tensor, outlier_idx: torch.Tensor,
+                       out: Optional[Quantized] = None, stream=None) -> Quantized:
+    """Offline weight quantization of fp16 W [N, K] (same encoding as the activations)."""
+    return _quant("atom_quant_weights", w, outlier_idx, out, stream)
+
+
+def atom_w4a4_gemm(qa: Quantized, qw: Quantized, K: int, y: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """Y fp16 [M, N] = sum_g sa*sw*P_g (see include/atom.h)."""
+    M, N = qa.rows, qw.rows
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=qa.q4.device)
+    st = lib().atom_w4a4_gemm(
+        _dev(qa.q4, torch.uint8, "qa4"), _dev(qa.q8, torch.int8, "qa8"),
+        _dev(qa.scales, torch.float32, "sa"), _dev(qw.q4, torch.uint8, "qw4"),
+        _dev(qw.q8, torch.int8, "qw8"), _dev(qw.scales, torch.float32, "sw"),
+        _dev(y, torch.float16, "y"), M, N, K, N_OUTLIER, GROUP, None, 0, _stream(stream))
+    _check("atom_w4a4_gemm", st)
+    return y
+
+
+def atom_w4a4_gemm_partials(qa: Quantized, qw: Quantized, K: int,
+                            partials: Optional[torch.Tensor] = None,
+                            y: Optional[torch.Tensor] = None, want_y: bool = True,
+                            stream=None):
+    """Debug entry: per-group int32 partial sums [G, M, N] (and Y unless want_y is False)."""
+    M, N = qa.rows, qw.rows
+    dev = qa.q4.device
+    if partials is None:
+        partials = torch.empty((K // GROUP, M, N), dtype=torch.int32, device=dev)
+    if want_y and y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    st = lib().atom_w4a4_gemm_partials(
+        _dev(qa.q4, torch.uint8, "qa4"), _dev(qa.q8, torch.int8, "qa8"),
+        _dev(qa.scales, torch.float32, "sa"), _dev(qw.q4, torch.uint8, "qw4"),
+        _dev(qw.q8, torch.int8, "qw8"), _dev(qw.scales, torch.float32, "sw"),
+        _dev(partials, torch.int32, "partials"),
+        _dev(y, torch.float16, "y") if want_y else None,
+        M, N, K, N_OUTLIER, GROUP, _stream(stream))
+    _check("atom_w4a4_gemm_partials", st)
+    return partials, y
+
+
+def atom_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().atom_gemm_workspace_bytes(M, N, K))
+
+
+def atom_device_status(clear: bool = True) -> int:
+    """First device-detected error since the last clear (0 = none); synchronises."""
+    return int(lib().atom_device_status(1 if clear else 0))
+
+
+def atom_status_string(status: int) -> str:
+    return lib().atom_status_string(status).decode()
+
+
+def atom_version() -> int:
+    return int(lib().atom_version())

@@ -1,0 +1,271 @@
+// atom_lib.cu -- the C ABI declared in include/atom.h: host-side argument
+// checks, tensor-map encoding and kernel launches. No allocation, no host
+// synchronisation on any compute entry point.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "atom.h"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxK = 32768;  // the permutation is staged as uint16 in shared memory
+
+struct DeviceState {
+  bool probed = false;
+  bool supported = false;
+  int sm_count = 0;
+  int smem_optin = 0;
+  bool gemm_attr[2] = {false, false};
+  uint32_t quant_smem_set = 0;
+};
+
+DeviceState g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+atom_status_t current_device(DeviceState **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATOM_ERR_CUDA;
+  DeviceState &d = g_devices[dev];
+  if (!d.probed) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!d.probed) {
+      int major = 0, minor = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+              cudaSuccess)
+        return ATOM_ERR_CUDA;
+      d.supported = (major == 10 && minor == 0);  // built for sm_100a only
+      d.probed = true;
+    }
+  }
+  if (!d.supported) return ATOM_ERR_UNSUPPORTED;
+  *out = &d;
+  return ATOM_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+atom_status_t check_method_params(int64_t K, int32_t n_outlier, int32_t group) {
+  if (group != 128 || n_outlier != 128) return ATOM_ERR_UNSUPPORTED;
+  if (K % 128 != 0 || K < 256 || K > kMaxK) return ATOM_ERR_SHAPE;
+  return ATOM_OK;
+}
+
+// ---------------------------------------------------------------- quantizer
+
+atom_status_t launch_quant(const void *x, int64_t rows, int64_t K, int64_t ld,
+                           const int32_t *idx, int32_t n_outlier, int32_t group, uint8_t *q4,
+                           int8_t *q8, float *scales, atom_stream_t stream) {
+  if (rows < 0 || ld < 0) return ATOM_ERR_INVALID_ARG;
+  atom_status_t st = check_method_params(K, n_outlier, group);
+  if (st != ATOM_OK) return st;
+  if (ld < K || ld % 8 != 0) return ATOM_ERR_SHAPE;
+  if (rows == 0) return ATOM_OK;
+  if (!x || !idx || !q4 || !q8 || !scales) return ATOM_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q4, 16) || !aligned(q8, 16) || !aligned(scales, 4) ||
+      !aligned(idx, 4))
+    return ATOM_ERR_ALIGN;
+
+  DeviceState *dev = nullptr;
+  if ((st = current_device(&dev)) != ATOM_OK) return st;
+
+  int stages = 3;
+  atomk::QuantLayout L = atomk::quant_layout(static_cast<int>(K), stages);
+  if (L.total > 110u * 1024u) {
+    stages = 2;
+    L = atomk::quant_layout(static_cast<int>(K), stages);
+  }
+  if (static_cast<int>(L.total) > dev->smem_optin) return ATOM_ERR_SHAPE;
+  if (dev->quant_smem_set < L.total) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (cudaFuncSetAttribute(atomk::reorder_quant_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(L.total)) != cudaSuccess)
+      return ATOM_ERR_CUDA;
+    dev->quant_smem_set = L.total;
+  }
+  // CTAs per SM: limited by 2048 threads and ~228 KB of shared memory (1 KB reserved per CTA).
+  int per_sm = static_cast<int>((228u * 1024u) / (L.total + 1024u));
+  per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+  const int64_t want = static_cast<int64_t>(per_sm) * dev->sm_count;
+  const int grid = static_cast<int>(rows < want ? rows : want);
+  atomk::reorder_quant_kernel<<<grid, atomk::kQuantThreads, L.total,
+                                reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __half *>(x), rows, static_cast<int>(K), ld, idx, q4, q8, scales, stages);
+  return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- GEMM
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Tensor map over an int8 [rows][128] matrix, boxes of box_rows x 128 bytes,
+// 128-byte swizzle (the K-major layout tcgen05 reads), zero fill past `rows`.
+bool encode_rows128(CUtensorMap *map, const void *base, int64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa,
+                          const uint8_t *qw4, const int8_t *qw8, const float *sw, void *y,
+                          int32_t *partials, int64_t M, int64_t N, int64_t K, int32_t n_outlier,
+                          int32_t group, atom_stream_t stream) {
+  if (M < 0 || N < 0) return ATOM_ERR_INVALID_ARG;
+  atom_status_t st = check_method_params(K, n_outlier, group);
+  if (st != ATOM_OK) return st;
+  if (N < 8 || N % 8 != 0 || M > INT32_MAX || N > INT32_MAX) return ATOM_ERR_SHAPE;
+  if (M == 0) return ATOM_OK;
+  if (!qa4 || !qa8 || !sa || !qw4 || !qw8 || !sw || (!y && !partials))
+    return ATOM_ERR_INVALID_ARG;
+  if (!aligned(qa4, 16) || !aligned(qa8, 16) || !aligned(qw4, 16) || !aligned(qw8, 16) ||
+      !aligned(sa, 4) || !aligned(sw, 4) || (y && !aligned(y, 16)) ||
+      (partials && !aligned(partials, 16)))
+    return ATOM_ERR_ALIGN;
+
+  DeviceState *dev = nullptr;
+  if ((st = current_device(&dev)) != ATOM_OK) return st;
+
+  using namespace atomk::gemm_cfg;
+  const bool pmode = partials != nullptr;
+  if (!dev->gemm_attr[pmode]) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    cudaError_t e = pmode ? cudaFuncSetAttribute(atomk::w4a4_gemm_kernel<true>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(kSmemBytes))
+                          : cudaFuncSetAttribute(atomk::w4a4_gemm_kernel<false>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return ATOM_ERR_CUDA;
+    dev->gemm_attr[pmode] = true;
+  }
+
+  CUtensorMap ta, tw;
+  if (!encode_rows128(&ta, qa8, M, BM) || !encode_rows128(&tw, qw8, N, BN)) return ATOM_ERR_CUDA;
+
+  atomk::GemmParams p;
+  p.qa4 = qa4;
+  p.sa = sa;
+  p.qw4 = qw4;
+  p.sw = sw;
+  p.y = static_cast<__half *>(y);
+  p.partials = partials;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.G = static_cast<int>(K / 128);
+  p.m_tiles = static_cast<int>((M + BM - 1) / BM);
+  p.n_tiles = static_cast<int>((N + BN - 1) / BN);
+  const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
+  if (tiles > INT32_MAX) return ATOM_ERR_SHAPE;
+  p.tiles = static_cast<int>(tiles);
+  const int grid = static_cast<int>(tiles < dev->sm_count ? tiles : dev->sm_count);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (pmode)
+    atomk::w4a4_gemm_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(ta, tw, p);
+  else
+    atomk::w4a4_gemm_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(ta, tw, p);
+  return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+atom_status_t atom_reorder_quant(const void *x, int64_t M, int64_t K, int64_t ld_x,
+                                 const int32_t *outlier_idx, int32_t n_outlier, int32_t group,
+                                 uint8_t *q4, int8_t *q8, float *scales, atom_stream_t stream) {
+  return launch_quant(x, M, K, ld_x, outlier_idx, n_outlier, group, q4, q8, scales, stream);
+}
+
+atom_status_t atom_quant_weights(const void *w, int64_t N, int64_t K, int64_t ld_w,
+                                 const int32_t *outlier_idx, int32_t n_outlier, int32_t group,
+                                 uint8_t *qw4, int8_t *qw8, float *sw, atom_stream_t stream) {
+  return launch_quant(w, N, K, ld_w, outlier_idx, n_outlier, group, qw4, qw8, sw, stream);
+}
+
+atom_status_t atom_w4a4_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa,
+                             const uint8_t *qw4, const int8_t *qw8, const float *sw, void *y,
+                             int64_t M, int64_t N, int64_t K, int32_t n_outlier, int32_t group,
+                             void *workspace, size_t workspace_bytes, atom_stream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!y && M > 0) return ATOM_ERR_INVALID_ARG;
+  return launch_gemm(qa4, qa8, sa, qw4, qw8, sw, y, nullptr, M, N, K, n_outlier, group, stream);
+}
+
+atom_status_t atom_w4a4_gemm_partials(const uint8_t *qa4, const int8_t *qa8, const float *sa,
+                                      const uint8_t *qw4, const int8_t *qw8, const float *sw,
+                                      int32_t *partials, void *y, int64_t M, int64_t N, int64_t K,
+                                      int32_t n_outlier, int32_t group, atom_stream_t stream) {
+  if (!partials && M > 0) return ATOM_ERR_INVALID_ARG;
+  return launch_gemm(qa4, qa8, sa, qw4, qw8, sw, y, partials, M, N, K, n_outlier, group, stream);
+}
+
+size_t atom_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  (void)M;
+  (void)N;
+  (void)K;
+  return 0;
+}
+
+atom_status_t atom_device_status(int clear) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATOM_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, atomk::g_device_status, sizeof(int)) != cudaSuccess)
+    return ATOM_ERR_CUDA;
+  if (clear) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(atomk::g_device_status, &zero, sizeof(int)) != cudaSuccess)
+      return ATOM_ERR_CUDA;
+  }
+  return static_cast<atom_status_t>(v);
+}
+
+const char *atom_status_string(atom_status_t status) {
+  switch (status) {
+    case ATOM_OK: return "ATOM_OK";
+    case ATOM_ERR_INVALID_ARG: return "ATOM_ERR_INVALID_ARG";
+    case ATOM_ERR_SHAPE: return "ATOM_ERR_SHAPE";
+    case ATOM_ERR_ALIGN: return "ATOM_ERR_ALIGN";
+    case ATOM_ERR_UNSUPPORTED: return "ATOM_ERR_UNSUPPORTED";
+    case ATOM_ERR_CUDA: return "ATOM_ERR_CUDA";
+    case ATOM_ERR_TIMEOUT: return "ATOM_ERR_TIMEOUT";
+  }
+  return "ATOM_ERR_UNKNOWN";
+}
+
+int atom_version(void) { return 100; }
+
+}  // extern "C"
