@@ -168,6 +168,8 @@ def main():
                     help="seconds of CPU oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--m", type=int, default=None,
+                    help="use only the first M activation rows (small profiling cases)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -176,6 +178,9 @@ def main():
 
     from w4a4_mixed_precision_b200 import inputs
     w = inputs.workload(args.workload)
+    if args.m is not None:
+        import dataclasses
+        w = dataclasses.replace(w, M=args.m, name=f"{w.name}_m{args.m}")
     workload_cfg = {"workload": f"{w.name} M={w.M} N={w.N} K={w.K}", "M": w.M, "N": w.N, "K": w.K,
                     "group": 128, "n_outlier": 128, "activations": w.describe(),
                     "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU",
@@ -198,7 +203,7 @@ def main():
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    A_h = inputs.activations(args.workload)
+    A_h = inputs.activations(args.workload, rows=w.M)
     W_h = inputs.weights(args.workload)
     idx_h = inputs.outlier_channels(args.workload)
 
@@ -374,7 +379,7 @@ def run_reference(args, w, workload_cfg, rank):
     from oracle import c_oracle
     cores = len(os.sched_getaffinity(0))
     c_oracle.set_threads(cores)
-    A = inputs.activations(args.workload)
+    A = inputs.activations(args.workload, rows=w.M)
     W = inputs.weights(args.workload)
     idx = inputs.outlier_channels(args.workload)
     qw = c_oracle.quantize(W, idx)
