@@ -21,6 +21,7 @@ struct DeviceState {
   int sm_count = 0;
   int smem_optin = 0;
   bool gemm_attr[2] = {false, false};
+  int gemm_clusters[2] = {0, 0};  // co-resident CTA pairs of the GEMM kernel
   uint32_t quant_smem_set = 0;
 };
 
@@ -146,6 +147,9 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   atom_status_t st = check_method_params(K, n_outlier, group);
   if (st != ATOM_OK) return st;
   if (N < 8 || N % 8 != 0 || M > INT32_MAX || N > INT32_MAX) return ATOM_ERR_SHAPE;
+  // the kernel addresses each packed INT4 matrix with 32-bit byte offsets
+  const int64_t q4_row = (K - 128) / 2;
+  if (M * q4_row >= (int64_t(1) << 31) || N * q4_row >= (int64_t(1) << 31)) return ATOM_ERR_SHAPE;
   if (M == 0) return ATOM_OK;
   if (!qa4 || !qa8 || !sa || !qw4 || !qw8 || !sw || (!y && !partials))
     return ATOM_ERR_INVALID_ARG;
@@ -161,18 +165,31 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   const bool pmode = partials != nullptr;
   if (!dev->gemm_attr[pmode]) {
     std::lock_guard<std::mutex> lock(g_mutex);
-    cudaError_t e = pmode ? cudaFuncSetAttribute(atomk::w4a4_gemm_kernel<true>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(kSmemBytes))
-                          : cudaFuncSetAttribute(atomk::w4a4_gemm_kernel<false>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess) return ATOM_ERR_CUDA;
+    const void *fn = pmode ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<true>)
+                           : reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<false>);
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+      return ATOM_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * dev->sm_count, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg) != cudaSuccess || clusters < 1)
+      clusters = dev->sm_count / 2;
+    dev->gemm_clusters[pmode] = clusters;
     dev->gemm_attr[pmode] = true;
   }
 
   CUtensorMap ta, tw;
-  if (!encode_rows128(&ta, qa8, M, BM) || !encode_rows128(&tw, qw8, N, BN)) return ATOM_ERR_CUDA;
+  if (!encode_rows128(&ta, qa8, M, BM) || !encode_rows128(&tw, qw8, N, BW)) return ATOM_ERR_CUDA;
 
   atomk::GemmParams p;
   p.qa4 = qa4;
@@ -185,12 +202,13 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.G = static_cast<int>(K / 128);
-  p.m_tiles = static_cast<int>((M + BM - 1) / BM);
+  p.m_tiles = static_cast<int>((M + kPairM - 1) / kPairM);
   p.n_tiles = static_cast<int>((N + BN - 1) / BN);
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
   if (tiles > INT32_MAX) return ATOM_ERR_SHAPE;
   p.tiles = static_cast<int>(tiles);
-  const int grid = static_cast<int>(tiles < dev->sm_count ? tiles : dev->sm_count);
+  const int64_t pairs = tiles < dev->gemm_clusters[pmode] ? tiles : dev->gemm_clusters[pmode];
+  const int grid = static_cast<int>(2 * pairs);   // CTA pairs (cluster of 2)
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (pmode)
     atomk::w4a4_gemm_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(ta, tw, p);
