@@ -124,18 +124,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tensor map over an int8 [rows][128] matrix, boxes of box_rows x 128 bytes,
-// 128-byte swizzle (the K-major layout tcgen05 reads), zero fill past `rows`.
-bool encode_rows128(CUtensorMap *map, const void *base, int64_t rows, uint32_t box_rows) {
+// 2-D tensor map over a row-major matrix of `rows` rows, `cols` elements per
+// row and a row stride of `stride_bytes`, copied in boxes of box_rows x box_cols;
+// reads past the matrix edge fill with zeros.
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t cols,
+               uint64_t rows, uint64_t stride_bytes, uint32_t box_cols, uint32_t box_rows,
+               CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {128};
-  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {stride_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -188,8 +190,23 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
     dev->gemm_attr[pmode] = true;
   }
 
-  CUtensorMap ta, tw;
-  if (!encode_rows128(&ta, qa8, M, BM) || !encode_rows128(&tw, qw8, N, BW)) return ATOM_ERR_CUDA;
+  const int64_t G = K / 128;
+  atomk::GemmMaps maps;
+  const bool sa_by_tma = (M % 4) == 0;   // rows of sa must be 16-byte aligned for TMA
+  const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  if (!encode_2d(&maps.a4, u8, qa4, q4_row, M, q4_row, 64, BM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_2d(&maps.w4, u8, qw4, q4_row, N, q4_row, 64, BW, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_2d(&maps.a8, u8, qa8, 128, M, 128, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&maps.w8, u8, qw8, 128, N, 128, 128, BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&maps.sw, f32, sw, N, G, N * 4, BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return ATOM_ERR_CUDA;
+  if (sa_by_tma) {
+    if (!encode_2d(&maps.sa, f32, sa, M, G, M * 4, BM, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return ATOM_ERR_CUDA;
+  } else {
+    maps.sa = maps.sw;  // not used by the kernel
+  }
 
   atomk::GemmParams p;
   p.qa4 = qa4;
@@ -201,7 +218,8 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
-  p.G = static_cast<int>(K / 128);
+  p.G = static_cast<int>(G);
+  p.sa_by_tma = sa_by_tma ? 1 : 0;
   p.m_tiles = static_cast<int>((M + kPairM - 1) / kPairM);
   p.n_tiles = static_cast<int>((N + BN - 1) / BN);
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
@@ -211,9 +229,9 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   const int grid = static_cast<int>(2 * pairs);   // CTA pairs (cluster of 2)
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (pmode)
-    atomk::w4a4_gemm_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(ta, tw, p);
+    atomk::w4a4_gemm_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
   else
-    atomk::w4a4_gemm_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(ta, tw, p);
+    atomk::w4a4_gemm_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
   return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
 }
 

@@ -16,29 +16,29 @@
 // issues 2-SM MMAs (cta_group::2, M=256, N=256, K=32): CTA r holds A rows
 // [128r, 128r+128) and W rows [128r, 128r+128) of the tile in its shared
 // memory, and its TMEM receives output rows [128r, 128r+128) x 256 columns.
-// The pairs are persistent over tiles (m fastest). One pipeline step per
-// 128-wide K group, with these warp roles in each CTA:
+// The pairs are persistent over tiles (m fastest). One pipeline stage per
+// 128-wide K group, with these roles in each CTA:
 //
-//   loader warps 1..7  LDG the packed INT4 group (64 bytes per row) one group
-//                      ahead into registers, expand each nibble to a byte
+//   producer (warp 0, lane 0)  TMA copies of the group's packed INT4 tiles
+//                      (128 rows x 64 bytes of A and of W), or of the INT8
+//                      outlier tiles straight into MMA layout, plus the
+//                      group's sa and sw vectors, into a free stage.
+//   MMA issuer (warp 0, lane 0 of the leader CTA only) 4 x 2-SM MMA into one
+//                      of two TMEM accumulators (2 x 256 int32 columns per
+//                      CTA), then commits to both CTAs' "stage empty" and
+//                      "accumulator full" barriers.
+//   unpack warps 1..7  expand each nibble of the staged packed tiles to a byte
 //                      holding 16*q (x << 4 & 0xF0 / x & 0xF0), store K-major
-//                      with the 128-byte swizzle, plus the group's scales. For
-//                      the INT8 outlier group one thread issues two TMA tile
-//                      loads instead. Every loader warp arrives on the pair
-//                      leader's "operands full" barrier.
-//   MMA warp 0         (leader CTA only) 4 x 2-SM MMA into one of two TMEM
-//                      accumulators (2 x 256 int32 columns per CTA), then
-//                      commits to both CTAs' "stage empty" and "accumulator
-//                      full" barriers.
+//                      with the 128-byte swizzle, and lay the scales out for
+//                      the drain; then arrive on the leader's "operands ready".
 //   drain warps 8..15  read the partials with the 16x256b TMEM shape (a thread
-//                      holds 4 rows x 2 columns of every 8-column block),
-//                      refill the accumulator with the conversion bias, and
-//                      accumulate sa*sw*P into fp32 registers. After the last
-//                      group of a tile: fp16 stores.
+//                      holds 4 rows x 2 columns of every 8-column block), release
+//                      the accumulator, and accumulate sa*sw*P into fp32
+//                      registers. After the last group of a tile: fp16 stores.
 //
-// Exact integer -> float: every accumulator starts at the bit pattern of
-// 1.5*2^23 (0x4B400000) and the MMAs add P on top, so the drain reads
-// F = 1.5*2^23 + P as a float with no integer instruction (|P| < 2^22).
+// Exact integer -> float: F = float with the bits P + 0x4B400000 equals
+// 1.5*2^23 + P exactly for |P| < 2^22 (one integer add per element; the
+// alternative of pre-filling TMEM with that bias doubles the TMEM traffic).
 // Dequantisation: with sw' = sw truncated to 22 significant bits, C*sw' is
 // exact for C = 1.5*2^23, so t = fma(F, sw', -C*sw') = round(P*sw') in one
 // instruction, then acc = fma(t, sa, acc); both run as packed f32x2 pairs.
@@ -60,28 +60,33 @@ constexpr int BM = 128;          // A rows per CTA (256 per pair)
 constexpr int BN = 256;          // output columns per pair tile
 constexpr int BW = 128;          // W rows per CTA
 constexpr int kPairM = 2 * BM;
-constexpr int kStages = 6;
+constexpr int kStages = 4;
 constexpr int kThreads = 512;
-constexpr int kLoaderThreads = 224;  // warps 1..7
-constexpr uint32_t kABytes = BM * 128;
-constexpr uint32_t kBBytes = BW * 128;
-constexpr uint32_t kSaOff = kABytes + kBBytes;
-constexpr uint32_t kSwOff = kSaOff + BM * 4;
-constexpr uint32_t kStageBytes = 34u * 1024u;
+constexpr int kUnpackThreads = 224;  // warps 1..7
+// stage layout (bytes from a 1024-aligned stage base)
+constexpr uint32_t kABytes = BM * 128;                 // unpacked / INT8 A, 128-byte swizzle
+constexpr uint32_t kBBytes = BW * 128;                 // unpacked / INT8 W, 128-byte swizzle
+constexpr uint32_t kPackAOff = kABytes + kBBytes;      // packed A, 128 rows x 64 B
+constexpr uint32_t kPackWOff = kPackAOff + BM * 64;    // packed W, 128 rows x 64 B
+constexpr uint32_t kSwLinOff = kPackWOff + BW * 64;    // sw as copied (256 floats)
+constexpr uint32_t kSaLinOff = kSwLinOff + BN * 4;     // sa as copied (128 floats)
+constexpr uint32_t kSwOff = kSaLinOff + BM * 4;        // sw in drain order
+constexpr uint32_t kSaOff = kSwOff + BN * 4;           // sa in drain order
+constexpr uint32_t kStageBytes = 52u * 1024u;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBarBytes = 1024;
 constexpr uint32_t kSmemBytes = kBarBytes + kStages * kStageBytes + 1024;  // + alignment slack
 constexpr int kPackedChunks = (BM + BW) * 4;                                   // 16-B chunks / group
-constexpr int kChunksPerThread = (kPackedChunks + kLoaderThreads - 1) / kLoaderThreads;
+constexpr int kChunksPerThread = (kPackedChunks + kUnpackThreads - 1) / kUnpackThreads;
 constexpr uint32_t kIdesc = idesc_i8(kPairM, BN);
 constexpr uint32_t kBias = 0x4B400000u;  // bits of 1.5 * 2^23
 constexpr float kBiasF = 12582912.0f;
-constexpr int kLoaderRegs = 80;
-constexpr int kDrainRegs = 176;
-static_assert(kSwOff + BN * 4 <= kStageBytes, "stage overflow");
+constexpr int kUnpackRegs = 56;
+constexpr int kDrainRegs = 200;
+static_assert(kSaOff + BM * 4 <= kStageBytes, "stage overflow");
 static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-static_assert(2 * 128 * (kLoaderRegs + kDrainRegs) == 65536, "register split must fill the file");
+static_assert(2 * 128 * (kUnpackRegs + kDrainRegs) == 65536, "register split must fill the file");
 }  // namespace gemm_cfg
 
 struct GemmParams {
@@ -93,15 +98,8 @@ struct GemmParams {
   int32_t *partials;   // partials mode only
   int M, N, K, G;
   int m_tiles, n_tiles, tiles;   // pair tiles of 256 x 256
+  int sa_by_tma;                 // M % 4 == 0: sa rows are 16-byte aligned for TMA
 };
-
-__device__ __forceinline__ uint4 ldg_stream_v4(const void *p) {
-  uint4 v;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-      : "l"(p));
-  return v;
-}
 
 // Predicated global stores. Keeping the predicate inside the instruction
 // (rather than branching around the store) keeps the epilogue one basic block,
@@ -148,49 +146,7 @@ __device__ __forceinline__ int64_t pair_iterations(const GemmParams &p) {
   return static_cast<int64_t>(mine) * p.G;
 }
 
-// ------------------------------------------------------------------ loader role
-
-struct LoaderRegs {
-  uint4 chunk[gemm_cfg::kChunksPerThread];
-  float sc[3];
-};
-
-// Packed chunk i (16 bytes) of this thread for group w.g, or zeros past the matrix edge.
-__device__ __forceinline__ uint4 loader_chunk(const GemmParams &p, const TileWalk &w, int rank,
-                                              int lt, int i) {
-  using namespace gemm_cfg;
-  const int c = lt + kLoaderThreads * i;
-  if (c >= kPackedChunks || w.g >= p.G - 1) return make_uint4(0u, 0u, 0u, 0u);
-  // byte offsets fit in 32 bits: the host limits each packed matrix to < 2 GiB
-  const uint32_t row_bytes = static_cast<uint32_t>(p.K - 128) / 2;
-  const bool is_a = c < BM * 4;
-  const int grow = is_a ? w.m0 + BM * rank + (c >> 2) : w.n0 + BW * rank + ((c - BM * 4) >> 2);
-  if (grow >= (is_a ? p.M : p.N)) return make_uint4(0u, 0u, 0u, 0u);
-  const uint32_t off =
-      static_cast<uint32_t>(grow) * row_bytes + static_cast<uint32_t>(w.g) * 64u + (c & 3) * 16u;
-  return ldg_stream_v4((is_a ? p.qa4 : p.qw4) + off);
-}
-
-// Scale k of this thread for group w.g: sa of row lt (lt < 128) or sw of column lt-128+96k.
-__device__ __forceinline__ float loader_scale(const GemmParams &p, const TileWalk &w, int rank,
-                                              int lt, int k) {
-  using namespace gemm_cfg;
-  if (lt < BM) {
-    const int m = w.m0 + BM * rank + lt;
-    return (k == 0 && m < p.M) ? __ldg(p.sa + static_cast<int64_t>(w.g) * p.M + m) : 0.f;
-  }
-  const int j = lt - BM + 96 * k;
-  const int n = w.n0 + j;
-  return (j < BN && n < p.N) ? __ldg(p.sw + static_cast<int64_t>(w.g) * p.N + n) : 0.f;
-}
-
-__device__ __forceinline__ void loader_fetch(const GemmParams &p, const TileWalk &w, int rank,
-                                             int lt, LoaderRegs &r) {
-#pragma unroll
-  for (int i = 0; i < gemm_cfg::kChunksPerThread; ++i) r.chunk[i] = loader_chunk(p, w, rank, lt, i);
-#pragma unroll
-  for (int k = 0; k < 3; ++k) r.sc[k] = loader_scale(p, w, rank, lt, k);
-}
+// ------------------------------------------------------------------ unpack role
 
 // Scale layouts in a stage, ordered for the drain's 16x256b fragments:
 //  sa: row r = 32q + i + 8k (i < 8, k < 4) at q*32 + i*4 + k, so a thread's four
@@ -204,60 +160,80 @@ __device__ __forceinline__ int sw_slot(int n) {
   return ((n >> 4) * 4 + ((w & 7) >> 1)) * 4 + ((w >> 3) << 1) + (w & 1);
 }
 
-// Expands and stores this thread's chunks and scales of group w.g into the stage,
-// reloading each register for group wn.g right after it has been stored (so
-// one group of loads stays in flight with a single set of registers).
-__device__ __forceinline__ void loader_store_refetch(const GemmParams &p, const TileWalk &w,
-                                                     const TileWalk &wn, bool refetch, int rank,
-                                                     int lt, LoaderRegs &r, uint8_t *stage) {
+// Expands this thread's share of the staged packed tiles into the swizzled
+// MMA operands and lays out the scales. `sa_direct` is this thread's sa value
+// when sa does not come through TMA (rows not 16-byte aligned).
+__device__ __forceinline__ void unpack_stage(const GemmParams &p, const TileWalk &w, int lt,
+                                             uint8_t *stage, float sa_direct) {
   using namespace gemm_cfg;
-  const bool int4_group = w.g < p.G - 1;
+  if (w.g < p.G - 1) {
 #pragma unroll
-  for (int i = 0; i < kChunksPerThread; ++i) {
-    const int c = lt + kLoaderThreads * i;
-    if (int4_group && c < kPackedChunks) {
-      const bool is_a = c < BM * 4;
-      const int cc = c & 3;
-      const int row = (is_a ? c : c - BM * 4) >> 2;
-      uint8_t *dst = stage + (is_a ? 0u : kABytes) + row * 128;
-      const uint4 v = r.chunk[i];
-      const uint4 lo = make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
-                                  (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
-      const uint4 hi = make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
-                                  v.w & 0xF0F0F0F0u);
-      const int sw = row & 7;
-      *reinterpret_cast<uint4 *>(dst + (((2 * cc) ^ sw) << 4)) = lo;
-      *reinterpret_cast<uint4 *>(dst + (((2 * cc + 1) ^ sw) << 4)) = hi;
+    for (int i = 0; i < kChunksPerThread; ++i) {
+      const int c = lt + kUnpackThreads * i;
+      if (c < kPackedChunks) {
+        const bool is_a = c < BM * 4;
+        const int cc = c & 3;
+        const int row = (is_a ? c : c - BM * 4) >> 2;
+        const uint4 v = *reinterpret_cast<const uint4 *>(
+            stage + (is_a ? kPackAOff : kPackWOff) + row * 64 + cc * 16);
+        uint8_t *dst = stage + (is_a ? 0u : kABytes) + row * 128;
+        const uint4 lo = make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
+                                    (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
+        const uint4 hi = make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
+                                    v.w & 0xF0F0F0F0u);
+        const int sw = row & 7;
+        *reinterpret_cast<uint4 *>(dst + (((2 * cc) ^ sw) << 4)) = lo;
+        *reinterpret_cast<uint4 *>(dst + (((2 * cc + 1) ^ sw) << 4)) = hi;
+      }
     }
-    if (refetch) r.chunk[i] = loader_chunk(p, wn, rank, lt, i);
   }
-  float *sa_s = reinterpret_cast<float *>(stage + kSaOff);
-  float *sw_s = reinterpret_cast<float *>(stage + kSwOff);
+  if (lt < BM) {
+    const float v = p.sa_by_tma ? reinterpret_cast<const float *>(stage + kSaLinOff)[lt] : sa_direct;
+    reinterpret_cast<float *>(stage + kSaOff)[sa_slot(lt)] = v;
+  } else {
 #pragma unroll
-  for (int k = 0; k < 3; ++k) {
-    if (lt < BM) {
-      if (k == 0) sa_s[sa_slot(lt)] = r.sc[0];
-    } else {
+    for (int k = 0; k < 3; ++k) {
       const int j = lt - BM + 96 * k;
-      if (j < BN) sw_s[sw_slot(j)] = __uint_as_float(__float_as_uint(r.sc[k]) & 0xFFFFFFFCu);
+      if (j < BN) {
+        const float v = reinterpret_cast<const float *>(stage + kSwLinOff)[j];
+        reinterpret_cast<float *>(stage + kSwOff)[sw_slot(j)] =
+            __uint_as_float(__float_as_uint(v) & 0xFFFFFFFCu);
+      }
     }
-    if (refetch) r.sc[k] = loader_scale(p, wn, rank, lt, k);
   }
+}
+
+// sa of this thread's row for group w.g read directly from global memory (only
+// used when M % 4 != 0, where the rows of sa are not 16-byte aligned for TMA).
+__device__ __forceinline__ float sa_direct_load(const GemmParams &p, const TileWalk &w, int rank,
+                                                int lt) {
+  const int m = w.m0 + gemm_cfg::BM * rank + lt;
+  return (lt < gemm_cfg::BM && m < p.M) ? __ldg(p.sa + static_cast<int64_t>(w.g) * p.M + m) : 0.f;
 }
 
 // ------------------------------------------------------------------ kernel
 
+// Tensor maps of the operands (built on the host for each call).
+struct GemmMaps {
+  CUtensorMap a4;   // packed INT4 A: uint8 [M][(K-128)/2], boxes of 128 rows x 64 bytes
+  CUtensorMap w4;   // packed INT4 W: uint8 [N][(K-128)/2], boxes of 128 rows x 64 bytes
+  CUtensorMap a8;   // INT8 A: [M][128], boxes 128 x 128 bytes, 128-byte swizzle
+  CUtensorMap w8;   // INT8 W: [N][128], boxes 128 x 128 bytes, 128-byte swizzle
+  CUtensorMap sa;   // fp32 [G][M], boxes of 1 x 128 (used when M % 4 == 0)
+  CUtensorMap sw;   // fp32 [G][N], boxes of 1 x 256
+};
+
 template <bool kPartials>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::kThreads, 1)
-w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a8,
-                 const __grid_constant__ CUtensorMap tmap_w8, const GemmParams p) {
+w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   using namespace gemm_cfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
 
-  uint64_t *lfull = reinterpret_cast<uint64_t *>(smem);  // [kStages] local loaders -> drain
-  uint64_t *mfull = lfull + kStages;   // [kStages] leader's: both CTAs' loaders -> MMA
-  uint64_t *empty = mfull + kStages;   // [kStages] MMA commit + local drain -> loaders
+  uint64_t *pfull = reinterpret_cast<uint64_t *>(smem);  // [kStages] TMA -> unpackers (local)
+  uint64_t *lfull = pfull + kStages;   // [kStages] unpackers -> drain (local)
+  uint64_t *mfull = lfull + kStages;   // [kStages] leader's: both CTAs' unpackers -> MMA
+  uint64_t *empty = mfull + kStages;   // [kStages] MMA commit + local drain -> producer
   uint64_t *tfull = empty + kStages;   // [2]       MMA commit -> drain
   uint64_t *tempty = tfull + 2;        // [2]       leader's: both CTAs' drains -> MMA
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
@@ -269,8 +245,9 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a8,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&lfull[s], 7);       // local loader warps
-      mbar_init(&mfull[s], 14);      // loader warps of both CTAs
+      mbar_init(&pfull[s], 1);       // producer's expect_tx arrival (+ TMA bytes)
+      mbar_init(&lfull[s], 7);       // local unpack warps
+      mbar_init(&mfull[s], 14);      // unpack warps of both CTAs
       mbar_init(&empty[s], 1 + 8);   // MMA commit + local drain warps
     }
     for (int b = 0; b < 2; ++b) {
@@ -306,22 +283,6 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a8,
     const uint32_t tempty_leader0 = cluster_map(&tempty[0], 0);
     const uint32_t tempty_leader1 = cluster_map(&tempty[1], 0);
 
-    // Both accumulators start at the conversion bias.
-#pragma unroll 1
-    for (int b = 0; b < 2; ++b)
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        tmem_st_16x256b_x2_fill(tbase + lane_base + (static_cast<uint32_t>(16 * (c & 1)) << 16) +
-                                    b * BN + h * 128 + 16 * (c >> 1),
-                                kBias);
-    tmem_st_wait();
-    tc_fence_before_sync();
-    __syncwarp();
-    if (lane == 0) {
-      mbar_arrive_cluster(tempty_leader0);
-      mbar_arrive_cluster(tempty_leader1);
-    }
-
     float2 acc[64];
 #pragma unroll
     for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
@@ -347,157 +308,189 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a8,
       const float *sw_s = reinterpret_cast<const float *>(stage + kSwOff);
       const uint32_t tcol = tbase + lane_base + b * BN + h * 128;
 
-      // chunk c: 16-column block pair j = c >> 1, TMEM lane half lh = c & 1
-      uint32_t ra[8], rb[8];
-      tmem_ld_16x256b_x2(tcol, ra);
+      // chunk c: 32 columns j4 = c >> 1 of this half, TMEM lane half lh = c & 1
+      uint32_t ra[16], rb[16];
+      tmem_ld_16x256b_x4(tcol, ra);
       tmem_ld_wait(ra);
 #pragma unroll
-      for (int c = 0; c < 16; c += 2) {
-        const int j = c >> 1;
-        const float4 s4 = *reinterpret_cast<const float4 *>(sw_s + ((8 * h + j) * 4 + t0) * 4);
-        const float2 swa = make_float2(s4.x, s4.y), swb = make_float2(s4.z, s4.w);
-        const float2 nca = f2_mul(swa, negC), ncb = f2_mul(swb, negC);
+      for (int c = 0; c < 8; c += 2) {
+        const int j4 = c >> 1;
+        const float4 s4a = *reinterpret_cast<const float4 *>(sw_s + ((8 * h + 2 * j4) * 4 + t0) * 4);
+        const float4 s4b =
+            *reinterpret_cast<const float4 *>(sw_s + ((8 * h + 2 * j4 + 1) * 4 + t0) * 4);
+        const float2 swk[4] = {make_float2(s4a.x, s4a.y), make_float2(s4a.z, s4a.w),
+                               make_float2(s4b.x, s4b.y), make_float2(s4b.z, s4b.w)};
+        float2 nck[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) nck[k] = f2_mul(swk[k], negC);
 #pragma unroll
         for (int lh = 0; lh < 2; ++lh) {
-          uint32_t(&r)[8] = lh ? rb : ra;
-          uint32_t(&rn)[8] = lh ? ra : rb;
+          uint32_t(&r)[16] = lh ? rb : ra;
+          uint32_t(&rn)[16] = lh ? ra : rb;
           const int cn = c + lh + 1;  // next chunk
-          if (cn < 16)
-            tmem_ld_16x256b_x2(
-                tcol + (static_cast<uint32_t>(16 * (cn & 1)) << 16) + 16 * (cn >> 1), rn);
-          // this chunk's partials are in registers: refill it with the bias
-          tmem_st_16x256b_x2_fill(tcol + (static_cast<uint32_t>(16 * lh) << 16) + 16 * j, kBias);
+          if (cn < 8)
+            tmem_ld_16x256b_x4(
+                tcol + (static_cast<uint32_t>(16 * (cn & 1)) << 16) + 32 * (cn >> 1), rn);
+          if (cn == 8) {
+            // every column of this accumulator is in registers: hand it back
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(b ? tempty_leader1 : tempty_leader0);
+          }
           if (kPartials) {
             const int row0 = w.m0 + BM * rank + 32 * q + 16 * lh + i0;
-            const int col = w.n0 + h * 128 + 16 * j + 2 * t0;
             const bool int4_group = w.g < p.G - 1;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int row = row0 + 8 * (e & 1);
-              const int cc = col + 8 * (e >> 1);
-              int32_t v0 = static_cast<int32_t>(r[2 * e] - kBias);
-              int32_t v1 = static_cast<int32_t>(r[2 * e + 1] - kBias);
-              if (int4_group) {
-                v0 >>= 8;
-                v1 >>= 8;
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+              for (int v = 0; v < 2; ++v) {
+                const int row = row0 + 8 * v;
+                const int col = w.n0 + h * 128 + 32 * j4 + 8 * k + 2 * t0;
+                int32_t v0 = static_cast<int32_t>(r[4 * k + 2 * v]);
+                int32_t v1 = static_cast<int32_t>(r[4 * k + 2 * v + 1]);
+                if (int4_group) {
+                  v0 >>= 8;
+                  v1 >>= 8;
+                }
+                const bool ok = row < p.M && col < p.N;
+                st_global_v2_if(
+                    p.partials + (static_cast<int64_t>(w.g) * p.M + (ok ? row : 0)) * p.N +
+                        (ok ? col : 0),
+                    static_cast<uint32_t>(v0), static_cast<uint32_t>(v1), ok);
               }
-              const bool ok = row < p.M && cc < p.N;
-              st_global_v2_if(
-                  p.partials + (static_cast<int64_t>(w.g) * p.M + (ok ? row : 0)) * p.N +
-                      (ok ? cc : 0),
-                  static_cast<uint32_t>(v0), static_cast<uint32_t>(v1), ok);
-            }
           }
-          float2 *a = acc + (2 * j + lh) * 4;
-          const float2 f0 = make_float2(__uint_as_float(r[0]), __uint_as_float(r[1]));
-          const float2 f1 = make_float2(__uint_as_float(r[2]), __uint_as_float(r[3]));
-          const float2 f2 = make_float2(__uint_as_float(r[4]), __uint_as_float(r[5]));
-          const float2 f3 = make_float2(__uint_as_float(r[6]), __uint_as_float(r[7]));
           const float sa_lo = lh ? sa4.z : sa4.x, sa_hi = lh ? sa4.w : sa4.y;
-          a[0] = f2_fma(f2_fma(f0, swa, nca), make_float2(sa_lo, sa_lo), a[0]);
-          a[1] = f2_fma(f2_fma(f1, swa, nca), make_float2(sa_hi, sa_hi), a[1]);
-          a[2] = f2_fma(f2_fma(f2, swb, ncb), make_float2(sa_lo, sa_lo), a[2]);
-          a[3] = f2_fma(f2_fma(f3, swb, ncb), make_float2(sa_hi, sa_hi), a[3]);
-          if (cn < 16) tmem_ld_wait(rn);
+          float2 *a = acc + (j4 * 2 + lh) * 8;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 flo = make_float2(__uint_as_float(r[4 * k] + kBias),
+                                           __uint_as_float(r[4 * k + 1] + kBias));
+            const float2 fhi = make_float2(__uint_as_float(r[4 * k + 2] + kBias),
+                                           __uint_as_float(r[4 * k + 3] + kBias));
+            a[2 * k] = f2_fma(f2_fma(flo, swk[k], nck[k]), make_float2(sa_lo, sa_lo), a[2 * k]);
+            a[2 * k + 1] =
+                f2_fma(f2_fma(fhi, swk[k], nck[k]), make_float2(sa_hi, sa_hi), a[2 * k + 1]);
+          }
+          if (cn < 8) tmem_ld_wait(rn);
         }
       }
-      // the accumulator is read and refilled with the bias: hand it back
-      tmem_st_wait();
-      tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_cluster(b ? tempty_leader1 : tempty_leader0);
-        mbar_arrive(&empty[s]);
-      }
+      if (lane == 0) mbar_arrive(&empty[s]);  // this stage's scales are no longer needed
 
       if (w.g == p.G - 1) {
         // epilogue: this thread's 4 rows x 32 columns as fp16 pairs
         const bool have_y = p.y != nullptr;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j4 = 0; j4 < 4; ++j4)
 #pragma unroll
           for (int lh = 0; lh < 2; ++lh)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int row = w.m0 + BM * rank + 32 * q + 16 * lh + i0 + 8 * (e & 1);
-              const int col = w.n0 + h * 128 + 16 * j + 2 * t0 + 8 * (e >> 1);
-              const bool ok = have_y && row < p.M && col < p.N;
-              const float2 v = acc[(2 * j + lh) * 4 + e];
-              st_global_b32_if(p.y + static_cast<int64_t>(ok ? row : 0) * p.N + (ok ? col : 0),
-                               pack_half2_rn(v.x, v.y), ok);
-            }
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+              for (int v = 0; v < 2; ++v) {
+                const int row = w.m0 + BM * rank + 32 * q + 16 * lh + i0 + 8 * v;
+                const int col = w.n0 + h * 128 + 32 * j4 + 8 * k + 2 * t0;
+                const bool ok = have_y && row < p.M && col < p.N;
+                const float2 val = acc[(j4 * 2 + lh) * 8 + 2 * k + v];
+                st_global_b32_if(p.y + static_cast<int64_t>(ok ? row : 0) * p.N + (ok ? col : 0),
+                                 pack_half2_rn(val.x, val.y), ok);
+              }
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
       }
     }
   } else {
-    regs_decrease<kLoaderRegs>();
+    regs_decrease<kUnpackRegs>();
     if (warp == 0) {
-      // ============================================================== MMA issuer (leader)
-      if (rank == 0 && lane == 0) {
-        int64_t last = -1;
-        for (int64_t it = 0; it < iters; ++it) {
-          const int s = static_cast<int>(it % kStages), b = static_cast<int>(it & 1);
-          if (!mbar_wait_cluster(&mfull[s], static_cast<uint32_t>((it / kStages) & 1),
-                                 abort_flag) ||
-              !mbar_wait_cluster(&tempty[b], static_cast<uint32_t>((it >> 1) & 1), abort_flag)) {
-            fail();
-            break;
+      // ============================================================== producer (+ MMA on the leader)
+      if (lane == 0) {
+        TileWalk wp;
+        wp.start(p);
+        int64_t produced = 0, last_mma = -1;
+        auto produce = [&]() -> bool {
+          const int64_t j = produced;
+          const int s = static_cast<int>(j % kStages);
+          if (!mbar_wait(&empty[s], static_cast<uint32_t>(((j / kStages) & 1) ^ 1), abort_flag))
+            return false;
+          uint8_t *stage = stages + s * kStageBytes;
+          const int arow = wp.m0 + BM * rank, wrow = wp.n0 + BW * rank;
+          const bool int4_group = wp.g < p.G - 1;
+          const uint32_t bytes = (int4_group ? (BM + BW) * 64u : kABytes + kBBytes) + BN * 4u +
+                                 (p.sa_by_tma ? BM * 4u : 0u);
+          mbar_arrive_expect_tx(&pfull[s], bytes);
+          if (int4_group) {
+            tma_load_2d(stage + kPackAOff, &maps.a4, wp.g * 64, arow, &pfull[s]);
+            tma_load_2d(stage + kPackWOff, &maps.w4, wp.g * 64, wrow, &pfull[s]);
+          } else {
+            tma_load_2d(stage, &maps.a8, 0, arow, &pfull[s]);
+            tma_load_2d(stage + kABytes, &maps.w8, 0, wrow, &pfull[s]);
           }
-          tc_fence_after_sync();
-          const uint32_t a_addr = smem_addr(stages + s * kStageBytes);
-          const uint64_t adesc = smem_desc_k_sw128(a_addr);
-          const uint64_t bdesc = smem_desc_k_sw128(a_addr + kABytes);
-          const uint32_t d = tbase + b * BN;
+          tma_load_2d(stage + kSwLinOff, &maps.sw, wp.n0, wp.g, &pfull[s]);
+          if (p.sa_by_tma) tma_load_2d(stage + kSaLinOff, &maps.sa, arow, wp.g, &pfull[s]);
+          ++produced;
+          wp.next(p);
+          return true;
+        };
+        bool ok = true;
+        while (ok && produced < iters && produced < kStages - 1) ok = produce();
+        for (int64_t it = 0; ok && it < iters; ++it) {
+          if (rank == 0) {
+            const int s = static_cast<int>(it % kStages), b = static_cast<int>(it & 1);
+            if (!mbar_wait_cluster(&mfull[s], static_cast<uint32_t>((it / kStages) & 1),
+                                   abort_flag) ||
+                !mbar_wait_cluster(&tempty[b], static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
+                                   abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+            const uint32_t a_addr = smem_addr(stages + s * kStageBytes);
+            const uint64_t adesc = smem_desc_k_sw128(a_addr);
+            const uint64_t bdesc = smem_desc_k_sw128(a_addr + kABytes);
+            const uint32_t d = tbase + b * BN;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, 1u);
-          tc_commit_pair_multicast(&empty[s], 0x3);
-          tc_commit_pair_multicast(&tfull[b], 0x3);
-          last = it;
+            for (int k = 0; k < 4; ++k)
+              mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
+            tc_commit_pair_multicast(&empty[s], 0x3);
+            tc_commit_pair_multicast(&tfull[b], 0x3);
+            last_mma = it;
+          }
+          if (produced < iters) ok = produce();
         }
+        if (!ok) fail();
         // nothing may still write TMEM when it is released
-        if (last >= 0)
-          (void)mbar_wait(&tfull[last & 1], static_cast<uint32_t>((last >> 1) & 1), nullptr);
+        if (last_mma >= 0)
+          (void)mbar_wait(&tfull[last_mma & 1], static_cast<uint32_t>((last_mma >> 1) & 1),
+                          nullptr);
+        // after an abort, let the tensor copies still in flight land
+        if (!ok)
+          for (int64_t j = (produced > kStages ? produced - kStages : 0); j < produced; ++j)
+            (void)mbar_wait(&pfull[j % kStages], static_cast<uint32_t>((j / kStages) & 1), nullptr);
       }
     } else {
-      // ============================================================== loaders
+      // ============================================================== unpackers
       const int lt = threadIdx.x - 32;
-      const int lwarp = warp - 1;
       TileWalk w;
       w.start(p);
-      LoaderRegs cur;
-      if (iters > 0) loader_fetch(p, w, rank, lt, cur);
-      int64_t last_tma = -1;
+      float sa_d = (!p.sa_by_tma && iters > 0) ? sa_direct_load(p, w, rank, lt) : 0.f;
       for (int64_t it = 0; it < iters; ++it) {
         const int s = static_cast<int>(it % kStages);
         TileWalk wn = w;
         wn.next(p);
-        if (!mbar_wait(&empty[s], static_cast<uint32_t>(((it / kStages) & 1) ^ 1), abort_flag)) {
+        if (!mbar_wait(&pfull[s], static_cast<uint32_t>((it / kStages) & 1), abort_flag)) {
           fail();
           break;
         }
         uint8_t *stage = stages + s * kStageBytes;
-        loader_store_refetch(p, w, wn, it + 1 < iters, rank, lt, cur, stage);
+        unpack_stage(p, w, lt, stage, sa_d);
+        if (!p.sa_by_tma && it + 1 < iters) sa_d = sa_direct_load(p, wn, rank, lt);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&lfull[s]);
-          const uint32_t leader_full = cluster_map(&mfull[s], 0);
-          if (w.g == p.G - 1 && lwarp == 0) {
-            mbar_arrive_expect_tx_cluster(leader_full, kABytes + kBBytes);
-            tma_load_2d_pair(stage, &tmap_a8, 0, w.m0 + BM * rank, leader_full);
-            tma_load_2d_pair(stage + kABytes, &tmap_w8, 0, w.n0 + BW * rank, leader_full);
-            last_tma = it;
-          } else {
-            mbar_arrive_cluster(leader_full);
-          }
+          mbar_arrive_cluster(cluster_map(&mfull[s], 0));
         }
         w = wn;
-      }
-      // after an abort, let this CTA's last tensor copy land before its memory is released
-      if (*abort_flag && lane == 0 && lwarp == 0 && last_tma >= 0) {
-        const int s = static_cast<int>(last_tma % kStages);
-        (void)mbar_wait(&empty[s], static_cast<uint32_t>((last_tma / kStages) & 1), nullptr);
       }
     }
   }
