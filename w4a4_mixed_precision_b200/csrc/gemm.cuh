@@ -23,11 +23,13 @@
 //                      (128 rows x 64 bytes of A and of W), or of the INT8
 //                      outlier tiles straight into MMA layout, plus the
 //                      group's sa and sw vectors, into a free stage.
-//   MMA issuer (warp 0, lane 0 of the leader CTA only) 4 x 2-SM MMA into one
-//                      of two TMEM accumulators (2 x 256 int32 columns per
-//                      CTA), then commits to both CTAs' "stage empty" and
-//                      "accumulator full" barriers.
-//   unpack warps 1..7  expand each nibble of the staged packed tiles to a byte
+//   warp 1, lane 0     leader CTA: issues 4 x 2-SM MMA into one of two TMEM
+//                      accumulators (2 x 256 int32 columns per CTA), then
+//                      commits to both CTAs' "stage empty" and "accumulator
+//                      full" barriers. Peer CTA: relays the peer's "operands
+//                      ready" and "accumulator drained" events to the leader,
+//                      so only one cross-SM arrival per event is made.
+//   unpack warps 2..7  expand each nibble of the staged packed tiles to a byte
 //                      holding 16*q (x << 4 & 0xF0 / x & 0xF0), store K-major
 //                      with the 128-byte swizzle, and lay the scales out for
 //                      the drain; then arrive on the leader's "operands ready".
@@ -62,7 +64,7 @@ constexpr int BW = 128;          // W rows per CTA
 constexpr int kPairM = 2 * BM;
 constexpr int kStages = 4;
 constexpr int kThreads = 512;
-constexpr int kUnpackThreads = 224;  // warps 1..7
+constexpr int kUnpackThreads = 192;  // warps 2..7
 // stage layout (bytes from a 1024-aligned stage base)
 constexpr uint32_t kABytes = BM * 128;                 // unpacked / INT8 A, 128-byte swizzle
 constexpr uint32_t kBBytes = BW * 128;                 // unpacked / INT8 W, 128-byte swizzle
@@ -108,6 +110,15 @@ __device__ __forceinline__ void st_global_b32_if(void *p, uint32_t a, bool pred)
   asm volatile(
       "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t@q st.global.b32 [%0], %1;\n\t}" ::"l"(p),
       "r"(a), "r"(static_cast<uint32_t>(pred))
+      : "memory");
+}
+
+__device__ __forceinline__ void st_global_v4_if(void *p, uint32_t a, uint32_t b, uint32_t c,
+                                                uint32_t d, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+      "@q st.global.v4.b32 [%0], {%1, %2, %3, %4};\n\t}" ::"l"(p),
+      "r"(a), "r"(b), "r"(c), "r"(d), "r"(static_cast<uint32_t>(pred))
       : "memory");
 }
 
@@ -191,9 +202,11 @@ __device__ __forceinline__ void unpack_stage(const GemmParams &p, const TileWalk
     const float v = p.sa_by_tma ? reinterpret_cast<const float *>(stage + kSaLinOff)[lt] : sa_direct;
     reinterpret_cast<float *>(stage + kSaOff)[sa_slot(lt)] = v;
   } else {
+    constexpr int kSwThreads = kUnpackThreads - BM;   // threads laying out sw
+    static_assert(kSwThreads > 0, "unpack threads must cover sa and sw");
 #pragma unroll
-    for (int k = 0; k < 3; ++k) {
-      const int j = lt - BM + 96 * k;
+    for (int k = 0; k < (BN + kSwThreads - 1) / kSwThreads; ++k) {
+      const int j = lt - BM + kSwThreads * k;
       if (j < BN) {
         const float v = reinterpret_cast<const float *>(stage + kSwLinOff)[j];
         reinterpret_cast<float *>(stage + kSwOff)[sw_slot(j)] =
@@ -231,11 +244,11 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
 
   uint64_t *pfull = reinterpret_cast<uint64_t *>(smem);  // [kStages] TMA -> unpackers (local)
-  uint64_t *lfull = pfull + kStages;   // [kStages] unpackers -> drain (local)
-  uint64_t *mfull = lfull + kStages;   // [kStages] leader's: both CTAs' unpackers -> MMA
+  uint64_t *lfull = pfull + kStages;   // [kStages] local unpackers -> drain, MMA, relay
+  uint64_t *mfull = lfull + kStages;   // [kStages] leader only: the peer's relayed "unpacked"
   uint64_t *empty = mfull + kStages;   // [kStages] MMA commit + local drain -> producer
   uint64_t *tfull = empty + kStages;   // [2]       MMA commit -> drain
-  uint64_t *tempty = tfull + 2;        // [2]       leader's: both CTAs' drains -> MMA
+  uint64_t *tempty = tfull + 2;        // [2]       local drain (+ leader: the peer's relay)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   uint8_t *stages = smem + kBarBytes;
@@ -246,13 +259,13 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&pfull[s], 1);       // producer's expect_tx arrival (+ TMA bytes)
-      mbar_init(&lfull[s], 7);       // local unpack warps
-      mbar_init(&mfull[s], 14);      // unpack warps of both CTAs
+      mbar_init(&lfull[s], 6);       // local unpack warps
+      mbar_init(&mfull[s], 1);       // the peer's relay (leader's copy is used)
       mbar_init(&empty[s], 1 + 8);   // MMA commit + local drain warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 16);     // drain warps of both CTAs
+      mbar_init(&tempty[b], rank == 0 ? 8 + 1 : 8);  // local drain warps (+ peer relay)
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -280,8 +293,6 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     const int t0 = lane & 3;          // column pair within an 8-column block
     const int i0 = lane >> 2;         // row within a group of 8 lanes
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-    const uint32_t tempty_leader0 = cluster_map(&tempty[0], 0);
-    const uint32_t tempty_leader1 = cluster_map(&tempty[1], 0);
 
     float2 acc[64];
 #pragma unroll
@@ -335,7 +346,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             // every column of this accumulator is in registers: hand it back
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(b ? tempty_leader1 : tempty_leader0);
+            if (lane == 0) mbar_arrive(&tempty[b]);
           }
           if (kPartials) {
             const int row0 = w.m0 + BM * rank + 32 * q + 16 * lh + i0;
@@ -378,23 +389,42 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       if (lane == 0) mbar_arrive(&empty[s]);  // this stage's scales are no longer needed
 
       if (w.g == p.G - 1) {
-        // epilogue: this thread's 4 rows x 32 columns as fp16 pairs
+        // epilogue. For each 32-column chunk and row, the 4 lanes with the same
+        // i0 hold 2 columns of each of the 4 8-column blocks; a 4x4 transpose
+        // across those lanes gives lane t0 all 8 columns of block t0, written
+        // as one 16-byte store.
         const bool have_y = p.y != nullptr;
 #pragma unroll
         for (int j4 = 0; j4 < 4; ++j4)
 #pragma unroll
           for (int lh = 0; lh < 2; ++lh)
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int v = 0; v < 2; ++v) {
+              uint32_t hb[4];
 #pragma unroll
-              for (int v = 0; v < 2; ++v) {
-                const int row = w.m0 + BM * rank + 32 * q + 16 * lh + i0 + 8 * v;
-                const int col = w.n0 + h * 128 + 32 * j4 + 8 * k + 2 * t0;
-                const bool ok = have_y && row < p.M && col < p.N;
+              for (int k = 0; k < 4; ++k) {
                 const float2 val = acc[(j4 * 2 + lh) * 8 + 2 * k + v];
-                st_global_b32_if(p.y + static_cast<int64_t>(ok ? row : 0) * p.N + (ok ? col : 0),
-                                 pack_half2_rn(val.x, val.y), ok);
+                hb[k] = pack_half2_rn(val.x, val.y);
               }
+              // round r: send block t0^r to lane t0^r, receive my block t0 from it
+              uint32_t o0 = hb[0], o1 = hb[1], o2 = hb[2], o3 = hb[3];
+#pragma unroll
+              for (int r = 1; r < 4; ++r) {
+                const int idx = t0 ^ r;
+                const uint32_t send =
+                    idx == 0 ? hb[0] : (idx == 1 ? hb[1] : (idx == 2 ? hb[2] : hb[3]));
+                const uint32_t got = __shfl_xor_sync(0xffffffffu, send, r);
+                o0 = idx == 0 ? got : o0;
+                o1 = idx == 1 ? got : o1;
+                o2 = idx == 2 ? got : o2;
+                o3 = idx == 3 ? got : o3;
+              }
+              const int row = w.m0 + BM * rank + 32 * q + 16 * lh + i0 + 8 * v;
+              const int col = w.n0 + h * 128 + 32 * j4 + 8 * t0;
+              const bool ok = have_y && row < p.M && col < p.N;
+              st_global_v4_if(p.y + static_cast<int64_t>(ok ? row : 0) * p.N + (ok ? col : 0),
+                              o0, o1, o2, o3, ok);
+            }
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
       }
@@ -402,16 +432,19 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   } else {
     regs_decrease<kUnpackRegs>();
     if (warp == 0) {
-      // ============================================================== producer (+ MMA on the leader)
+      // ============================================================== producer
       if (lane == 0) {
         TileWalk wp;
         wp.start(p);
-        int64_t produced = 0, last_mma = -1;
-        auto produce = [&]() -> bool {
-          const int64_t j = produced;
-          const int s = static_cast<int>(j % kStages);
-          if (!mbar_wait(&empty[s], static_cast<uint32_t>(((j / kStages) & 1) ^ 1), abort_flag))
-            return false;
+        int64_t produced = 0;
+        bool ok = true;
+        for (; produced < iters; ++produced, wp.next(p)) {
+          const int s = static_cast<int>(produced % kStages);
+          if (!mbar_wait(&empty[s], static_cast<uint32_t>(((produced / kStages) & 1) ^ 1),
+                         abort_flag)) {
+            ok = false;
+            break;
+          }
           uint8_t *stage = stages + s * kStageBytes;
           const int arow = wp.m0 + BM * rank, wrow = wp.n0 + BW * rank;
           const bool int4_group = wp.g < p.G - 1;
@@ -427,49 +460,71 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
           }
           tma_load_2d(stage + kSwLinOff, &maps.sw, wp.n0, wp.g, &pfull[s]);
           if (p.sa_by_tma) tma_load_2d(stage + kSaLinOff, &maps.sa, arow, wp.g, &pfull[s]);
-          ++produced;
-          wp.next(p);
-          return true;
-        };
-        bool ok = true;
-        while (ok && produced < iters && produced < kStages - 1) ok = produce();
-        for (int64_t it = 0; ok && it < iters; ++it) {
-          if (rank == 0) {
-            const int s = static_cast<int>(it % kStages), b = static_cast<int>(it & 1);
-            if (!mbar_wait_cluster(&mfull[s], static_cast<uint32_t>((it / kStages) & 1),
-                                   abort_flag) ||
-                !mbar_wait_cluster(&tempty[b], static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
-                                   abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after_sync();
-            const uint32_t a_addr = smem_addr(stages + s * kStageBytes);
-            const uint64_t adesc = smem_desc_k_sw128(a_addr);
-            const uint64_t bdesc = smem_desc_k_sw128(a_addr + kABytes);
-            const uint32_t d = tbase + b * BN;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
-            tc_commit_pair_multicast(&empty[s], 0x3);
-            tc_commit_pair_multicast(&tfull[b], 0x3);
-            last_mma = it;
-          }
-          if (produced < iters) ok = produce();
         }
-        if (!ok) fail();
+        if (!ok) {
+          fail();
+          // let the tensor copies still in flight land before shared memory is released
+          for (int64_t j = (produced > kStages ? produced - kStages : 0); j < produced; ++j)
+            (void)mbar_wait(&pfull[j % kStages], static_cast<uint32_t>((j / kStages) & 1), nullptr);
+        }
+      }
+    } else if (warp == 1) {
+      if (lane == 0 && rank == 0) {
+        // ============================================================ MMA issuer (leader)
+        int64_t last_mma = -1;
+        for (int64_t it = 0; it < iters; ++it) {
+          const int s = static_cast<int>(it % kStages), b = static_cast<int>(it & 1);
+          const uint32_t ph = static_cast<uint32_t>((it / kStages) & 1);
+          if (!mbar_wait(&lfull[s], ph, abort_flag) ||
+              !mbar_wait_cluster(&mfull[s], ph, abort_flag) ||
+              !mbar_wait_cluster(&tempty[b], static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
+                                 abort_flag)) {
+            fail();
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem_addr(stages + s * kStageBytes);
+          const uint64_t adesc = smem_desc_k_sw128(a_addr);
+          const uint64_t bdesc = smem_desc_k_sw128(a_addr + kABytes);
+          const uint32_t d = tbase + b * BN;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
+          tc_commit_pair_multicast(&empty[s], 0x3);
+          tc_commit_pair_multicast(&tfull[b], 0x3);
+          last_mma = it;
+        }
         // nothing may still write TMEM when it is released
         if (last_mma >= 0)
           (void)mbar_wait(&tfull[last_mma & 1], static_cast<uint32_t>((last_mma >> 1) & 1),
                           nullptr);
-        // after an abort, let the tensor copies still in flight land
-        if (!ok)
-          for (int64_t j = (produced > kStages ? produced - kStages : 0); j < produced; ++j)
-            (void)mbar_wait(&pfull[j % kStages], static_cast<uint32_t>((j / kStages) & 1), nullptr);
+      } else if (lane == 0) {
+        // ============================================================ relay (peer)
+        // One cross-SM arrival per event: "this CTA's operands of group it are
+        // unpacked" and "this CTA's accumulator of group it-1 is drained".
+        for (int64_t it = 0; it <= iters; ++it) {
+          if (it < iters) {
+            const int s = static_cast<int>(it % kStages);
+            if (!mbar_wait(&lfull[s], static_cast<uint32_t>((it / kStages) & 1), abort_flag)) {
+              fail();
+              break;
+            }
+            mbar_arrive_cluster(cluster_map(&mfull[s], 0));
+          }
+          if (it >= 1) {
+            const int64_t j = it - 1;
+            const int b = static_cast<int>(j & 1);
+            if (!mbar_wait(&tempty[b], static_cast<uint32_t>((j >> 1) & 1), abort_flag)) {
+              fail();
+              break;
+            }
+            mbar_arrive_cluster(cluster_map(&tempty[b], 0));
+          }
+        }
       }
     } else {
       // ============================================================== unpackers
-      const int lt = threadIdx.x - 32;
+      const int lt = threadIdx.x - 64;
       TileWalk w;
       w.start(p);
       float sa_d = (!p.sa_by_tma && iters > 0) ? sa_direct_load(p, w, rank, lt) : 0.f;
@@ -486,10 +541,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         if (!p.sa_by_tma && it + 1 < iters) sa_d = sa_direct_load(p, wn, rank, lt);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&lfull[s]);
-          mbar_arrive_cluster(cluster_map(&mfull[s], 0));
-        }
+        if (lane == 0) mbar_arrive(&lfull[s]);
         w = wn;
       }
     }
