@@ -12,31 +12,35 @@
 // 4-bit integer MMA, so both the INT4 groups and the INT8 outlier group run on
 // tcgen05.mma kind::i8.
 //
-// Structure. A cluster of two CTAs on two SMs owns a 256x256 output tile and
-// issues 2-SM MMAs (cta_group::2, M=256, N=256, K=32): CTA r holds A rows
-// [128r, 128r+128) and W rows [128r, 128r+128) of the tile in its shared
-// memory, and its TMEM receives output rows [128r, 128r+128) x 256 columns.
-// The pairs are persistent over tiles (m fastest). One pipeline stage per
-// 128-wide K group, with these roles in each CTA:
+// Structure. A cluster of two CTAs on two SMs owns a 256x256 output tile: CTA
+// r holds A rows [128r, 128r+128) and W rows [128r, 128r+128) of the tile in
+// its shared memory, and its TMEM receives output rows [128r, 128r+128). Each
+// 128-wide K group is issued as two column halves of 2-SM MMAs (cta_group::2,
+// M=256, N=128, K=32); half h takes W rows [64h, 64h+64) from each CTA, so
+// accumulator column j of half h is tile column 64h + (j mod 64) + 128*(j/64).
+// Two groups in flight x two halves gives four 128-column accumulators per
+// CTA, and the drain hands each half back as soon as it has read it, so the
+// tensor cores never wait for a whole group to be drained. The pairs are
+// persistent over tiles (m fastest). Roles in each CTA:
 //
 //   producer (warp 0, lane 0)  TMA copies of the group's packed INT4 tiles
 //                      (128 rows x 64 bytes of A and of W), or of the INT8
 //                      outlier tiles straight into MMA layout, plus the
 //                      group's sa and sw vectors, into a free stage.
-//   warp 1, lane 0     leader CTA: issues 4 x 2-SM MMA into one of two TMEM
-//                      accumulators (2 x 256 int32 columns per CTA), then
-//                      commits to both CTAs' "stage empty" and "accumulator
-//                      full" barriers. Peer CTA: relays the peer's "operands
-//                      ready" and "accumulator drained" events to the leader,
-//                      so only one cross-SM arrival per event is made.
+//   warp 1, lane 0     (leader CTA) per group and half: 4 x 2-SM MMA into a
+//                      128-column TMEM accumulator, commit to both CTAs' "half
+//                      full" barrier; after both halves commit to both CTAs'
+//                      "stage empty" barrier.
 //   unpack warps 2..7  expand each nibble of the staged packed tiles to a byte
 //                      holding 16*q (x << 4 & 0xF0 / x & 0xF0), store K-major
 //                      with the 128-byte swizzle, and lay the scales out for
-//                      the drain; then arrive on the leader's "operands ready".
+//                      the drain; then one thread signals "operands ready"
+//                      locally and, in the peer CTA, to the leader.
 //   drain warps 8..15  read the partials with the 16x256b TMEM shape (a thread
 //                      holds 4 rows x 2 columns of every 8-column block), release
-//                      the accumulator, and accumulate sa*sw*P into fp32
-//                      registers. After the last group of a tile: fp16 stores.
+//                      each half once read (one arrival per CTA, on the leader),
+//                      and accumulate sa*sw*P into fp32 registers. After the
+//                      last group of a tile: fp16 stores.
 //
 // Exact integer -> float: F = float with the bits P + 0x4B400000 equals
 // 1.5*2^23 + P exactly for |P| < 2^22 (one integer add per element; the
@@ -80,7 +84,8 @@ constexpr uint32_t kBarBytes = 1024;
 constexpr uint32_t kSmemBytes = kBarBytes + kStages * kStageBytes + 1024;  // + alignment slack
 constexpr int kPackedChunks = (BM + BW) * 4;                                   // 16-B chunks / group
 constexpr int kChunksPerThread = (kPackedChunks + kUnpackThreads - 1) / kUnpackThreads;
-constexpr uint32_t kIdesc = idesc_i8(kPairM, BN);
+constexpr int kHalfN = BN / 2;   // columns per MMA / accumulator half
+constexpr uint32_t kIdesc = idesc_i8(kPairM, kHalfN);
 constexpr uint32_t kBias = 0x4B400000u;  // bits of 1.5 * 2^23
 constexpr float kBiasF = 12582912.0f;
 constexpr int kUnpackRegs = 56;
@@ -159,12 +164,20 @@ __device__ __forceinline__ int64_t pair_iterations(const GemmParams &p) {
 
 // ------------------------------------------------------------------ unpack role
 
+// Tile column of accumulator column c (0..255): c = 128h + j holds the MMA half
+// h column j, which is W row 64h + (j mod 64) of CTA j/64.
+__device__ __forceinline__ int tile_col(int c) {
+  const int h = c >> 7, j = c & 127;
+  return ((j >> 6) << 7) + (h << 6) + (j & 63);
+}
+
 // Scale layouts in a stage, ordered for the drain's 16x256b fragments:
 //  sa: row r = 32q + i + 8k (i < 8, k < 4) at q*32 + i*4 + k, so a thread's four
 //      rows are one 16-byte load;
-//  sw: column n = 16S + 8u + 2t + e (t < 4, e, u < 2) at (4S + t)*4 + 2u + e, so a
-//      thread's four columns of a 16-column block are one 16-byte load. The
-//      stored value is sw truncated to 22 significant bits.
+//  sw: accumulator column c = 16S + 8u + 2t + e (t < 4, e, u < 2) at
+//      (4S + t)*4 + 2u + e, so a thread's four columns of a 16-column block are
+//      one 16-byte load. The stored value is sw of tile column tile_col(c),
+//      truncated to 22 significant bits.
 __device__ __forceinline__ int sa_slot(int r) { return (r >> 5) * 32 + (r & 7) * 4 + ((r >> 3) & 3); }
 __device__ __forceinline__ int sw_slot(int n) {
   const int w = n & 15;
@@ -208,7 +221,7 @@ __device__ __forceinline__ void unpack_stage(const GemmParams &p, const TileWalk
     for (int k = 0; k < (BN + kSwThreads - 1) / kSwThreads; ++k) {
       const int j = lt - BM + kSwThreads * k;
       if (j < BN) {
-        const float v = reinterpret_cast<const float *>(stage + kSwLinOff)[j];
+        const float v = reinterpret_cast<const float *>(stage + kSwLinOff)[tile_col(j)];
         reinterpret_cast<float *>(stage + kSwOff)[sw_slot(j)] =
             __uint_as_float(__float_as_uint(v) & 0xFFFFFFFCu);
       }
@@ -236,6 +249,9 @@ struct GemmMaps {
   CUtensorMap sw;   // fp32 [G][N], boxes of 1 x 256
 };
 
+// Hardware barrier ids for the role-internal gathers (0 is __syncthreads).
+constexpr uint32_t kBarDrain = 1, kBarUnpack = 2;
+
 template <bool kPartials>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::kThreads, 1)
 w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
@@ -243,13 +259,13 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
 
-  uint64_t *pfull = reinterpret_cast<uint64_t *>(smem);  // [kStages] TMA -> unpackers (local)
-  uint64_t *lfull = pfull + kStages;   // [kStages] local unpackers -> drain, MMA, relay
-  uint64_t *mfull = lfull + kStages;   // [kStages] leader only: the peer's relayed "unpacked"
+  uint64_t *pfull = reinterpret_cast<uint64_t *>(smem);  // [kStages] TMA -> unpackers
+  uint64_t *lfull = pfull + kStages;   // [kStages] unpacked (local) -> drain, MMA
+  uint64_t *mfull = lfull + kStages;   // [kStages] leader only: the peer's "unpacked"
   uint64_t *empty = mfull + kStages;   // [kStages] MMA commit + local drain -> producer
-  uint64_t *tfull = empty + kStages;   // [2]       MMA commit -> drain
-  uint64_t *tempty = tfull + 2;        // [2]       local drain (+ leader: the peer's relay)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  uint64_t *tfull = empty + kStages;   // [4]       accumulator (buffer b, half h) at 2b+h
+  uint64_t *tempty = tfull + 4;        // [4]       leader only: both CTAs drained (b, h)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 4);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   uint8_t *stages = smem + kBarBytes;
 
@@ -259,13 +275,13 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&pfull[s], 1);       // producer's expect_tx arrival (+ TMA bytes)
-      mbar_init(&lfull[s], 6);       // local unpack warps
-      mbar_init(&mfull[s], 1);       // the peer's relay (leader's copy is used)
+      mbar_init(&lfull[s], 1);       // one unpack thread after the unpack gather
+      mbar_init(&mfull[s], 1);       // the peer's unpack thread
       mbar_init(&empty[s], 1 + 8);   // MMA commit + local drain warps
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], rank == 0 ? 8 + 1 : 8);  // local drain warps (+ peer relay)
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 2);      // one drain thread of each CTA
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -288,11 +304,14 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   if (warp >= 8) {
     // ================================================================ drain
     regs_increase<kDrainRegs>();
-    const int q = warp & 3;           // TMEM lane quarter this warp may access
-    const int h = (warp - 8) >> 2;    // which 128-column half of the tile
+    const int dw = warp - 8;
+    const int q = dw & 3;             // TMEM lane quarter this warp may access
+    const int hh = dw >> 2;           // which 64 columns of each accumulator half
     const int t0 = lane & 3;          // column pair within an 8-column block
     const int i0 = lane >> 2;         // row within a group of 8 lanes
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    const bool releaser = dw == 0 && lane == 0;
+    const uint32_t tempty_leader = cluster_map(&tempty[0], 0);
 
     float2 acc[64];
 #pragma unroll
@@ -300,10 +319,13 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     const float2 negC = make_float2(-kBiasF, -kBiasF);
     TileWalk w;
     w.start(p);
-    for (int64_t it = 0; it < iters; ++it, w.next(p)) {
+    bool aborted = false;
+    for (int64_t it = 0; it < iters && !aborted; ++it, w.next(p)) {
       const int s = static_cast<int>(it % kStages), b = static_cast<int>(it & 1);
-      if (!mbar_wait(&tfull[b], static_cast<uint32_t>((it >> 1) & 1), abort_flag) ||
-          !mbar_wait(&lfull[s], static_cast<uint32_t>((it / kStages) & 1), abort_flag)) {
+      const uint32_t tph = static_cast<uint32_t>((it >> 1) & 1);
+      const bool ok = mbar_wait(&tfull[2 * b], tph, abort_flag) &&
+                      mbar_wait(&lfull[s], static_cast<uint32_t>((it / kStages) & 1), abort_flag);
+      if (named_bar_any(kBarDrain, 256, !ok)) {
         fail();
         break;
       }
@@ -317,74 +339,91 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         sa4.w *= 0.00390625f;
       }
       const float *sw_s = reinterpret_cast<const float *>(stage + kSwOff);
-      const uint32_t tcol = tbase + lane_base + b * BN + h * 128;
+      const uint32_t tbuf = tbase + lane_base + b * BN + hh * 64;
 
-      // chunk c: 32 columns j4 = c >> 1 of this half, TMEM lane half lh = c & 1
+      // chunk c = 4h + 2*j4 + lh: accumulator half h, 32 columns j4, TMEM lane half lh
       uint32_t ra[16], rb[16];
-      tmem_ld_16x256b_x4(tcol, ra);
+      tmem_ld_16x256b_x4(tbuf, ra);
       tmem_ld_wait(ra);
+      float2 swk[4], nck[4];
 #pragma unroll
-      for (int c = 0; c < 8; c += 2) {
-        const int j4 = c >> 1;
-        const float4 s4a = *reinterpret_cast<const float4 *>(sw_s + ((8 * h + 2 * j4) * 4 + t0) * 4);
-        const float4 s4b =
-            *reinterpret_cast<const float4 *>(sw_s + ((8 * h + 2 * j4 + 1) * 4 + t0) * 4);
-        const float2 swk[4] = {make_float2(s4a.x, s4a.y), make_float2(s4a.z, s4a.w),
-                               make_float2(s4b.x, s4b.y), make_float2(s4b.z, s4b.w)};
-        float2 nck[4];
+      for (int c = 0; c < 8; ++c) {
+        uint32_t(&r)[16] = (c & 1) ? rb : ra;
+        uint32_t(&rn)[16] = (c & 1) ? ra : rb;
+        const int h = c >> 2, j4 = (c >> 1) & 1, lh = c & 1;
+        const int c0 = h * 128 + hh * 64 + 32 * j4;   // accumulator column of this chunk
+        if (lh == 0) {
+          const float4 s4a = *reinterpret_cast<const float4 *>(sw_s + ((c0 >> 4) * 4 + t0) * 4);
+          const float4 s4b =
+              *reinterpret_cast<const float4 *>(sw_s + (((c0 >> 4) + 1) * 4 + t0) * 4);
+          swk[0] = make_float2(s4a.x, s4a.y);
+          swk[1] = make_float2(s4a.z, s4a.w);
+          swk[2] = make_float2(s4b.x, s4b.y);
+          swk[3] = make_float2(s4b.z, s4b.w);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) nck[k] = f2_mul(swk[k], negC);
-#pragma unroll
-        for (int lh = 0; lh < 2; ++lh) {
-          uint32_t(&r)[16] = lh ? rb : ra;
-          uint32_t(&rn)[16] = lh ? ra : rb;
-          const int cn = c + lh + 1;  // next chunk
-          if (cn < 8)
-            tmem_ld_16x256b_x4(
-                tcol + (static_cast<uint32_t>(16 * (cn & 1)) << 16) + 32 * (cn >> 1), rn);
-          if (cn == 8) {
-            // every column of this accumulator is in registers: hand it back
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[b]);
-          }
-          if (kPartials) {
-            const int row0 = w.m0 + BM * rank + 32 * q + 16 * lh + i0;
-            const bool int4_group = w.g < p.G - 1;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-#pragma unroll
-              for (int v = 0; v < 2; ++v) {
-                const int row = row0 + 8 * v;
-                const int col = w.n0 + h * 128 + 32 * j4 + 8 * k + 2 * t0;
-                int32_t v0 = static_cast<int32_t>(r[4 * k + 2 * v]);
-                int32_t v1 = static_cast<int32_t>(r[4 * k + 2 * v + 1]);
-                if (int4_group) {
-                  v0 >>= 8;
-                  v1 >>= 8;
-                }
-                const bool ok = row < p.M && col < p.N;
-                st_global_v2_if(
-                    p.partials + (static_cast<int64_t>(w.g) * p.M + (ok ? row : 0)) * p.N +
-                        (ok ? col : 0),
-                    static_cast<uint32_t>(v0), static_cast<uint32_t>(v1), ok);
-              }
-          }
-          const float sa_lo = lh ? sa4.z : sa4.x, sa_hi = lh ? sa4.w : sa4.y;
-          float2 *a = acc + (j4 * 2 + lh) * 8;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 flo = make_float2(__uint_as_float(r[4 * k] + kBias),
-                                           __uint_as_float(r[4 * k + 1] + kBias));
-            const float2 fhi = make_float2(__uint_as_float(r[4 * k + 2] + kBias),
-                                           __uint_as_float(r[4 * k + 3] + kBias));
-            a[2 * k] = f2_fma(f2_fma(flo, swk[k], nck[k]), make_float2(sa_lo, sa_lo), a[2 * k]);
-            a[2 * k + 1] =
-                f2_fma(f2_fma(fhi, swk[k], nck[k]), make_float2(sa_hi, sa_hi), a[2 * k + 1]);
-          }
-          if (cn < 8) tmem_ld_wait(rn);
+          for (int k = 0; k < 4; ++k) nck[k] = f2_mul(swk[k], negC);
         }
+        if (c == 3 || c == 7) {
+          // every chunk of half h is in registers: hand the half back
+          tc_fence_before_sync();
+          bool ok2 = true;
+          if (c == 3) ok2 = mbar_wait(&tfull[2 * b + 1], tph, abort_flag);
+          if (named_bar_any(kBarDrain, 256, !ok2)) {
+            fail();
+            aborted = true;
+            break;
+          }
+          if (releaser) {
+            if (rank == 0)
+              mbar_arrive(&tempty[2 * b + h]);
+            else
+              mbar_arrive_cluster_relaxed(tempty_leader + 8u * (2 * b + h));
+          }
+          if (c == 3) tc_fence_after_sync();
+        }
+        if (c + 1 < 8) {
+          const int cn = c + 1;
+          tmem_ld_16x256b_x4(tbase + lane_base + (static_cast<uint32_t>(16 * (cn & 1)) << 16) +
+                                 b * BN + (cn >> 2) * 128 + hh * 64 + 32 * ((cn >> 1) & 1),
+                             rn);
+        }
+        if (kPartials) {
+          const int row0 = w.m0 + BM * rank + 32 * q + 16 * lh + i0;
+          const bool int4_group = w.g < p.G - 1;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+              const int row = row0 + 8 * v;
+              const int col = w.n0 + tile_col(c0 + 8 * k + 2 * t0);
+              int32_t v0 = static_cast<int32_t>(r[4 * k + 2 * v]);
+              int32_t v1 = static_cast<int32_t>(r[4 * k + 2 * v + 1]);
+              if (int4_group) {
+                v0 >>= 8;
+                v1 >>= 8;
+              }
+              const bool okp = row < p.M && col < p.N;
+              st_global_v2_if(
+                  p.partials + (static_cast<int64_t>(w.g) * p.M + (okp ? row : 0)) * p.N +
+                      (okp ? col : 0),
+                  static_cast<uint32_t>(v0), static_cast<uint32_t>(v1), okp);
+            }
+        }
+        const float sa_lo = lh ? sa4.z : sa4.x, sa_hi = lh ? sa4.w : sa4.y;
+        float2 *a = acc + c * 8;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 flo = make_float2(__uint_as_float(r[4 * k] + kBias),
+                                         __uint_as_float(r[4 * k + 1] + kBias));
+          const float2 fhi = make_float2(__uint_as_float(r[4 * k + 2] + kBias),
+                                         __uint_as_float(r[4 * k + 3] + kBias));
+          a[2 * k] = f2_fma(f2_fma(flo, swk[k], nck[k]), make_float2(sa_lo, sa_lo), a[2 * k]);
+          a[2 * k + 1] =
+              f2_fma(f2_fma(fhi, swk[k], nck[k]), make_float2(sa_hi, sa_hi), a[2 * k + 1]);
+        }
+        if (c + 1 < 8) tmem_ld_wait(rn);
       }
+      if (aborted) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);  // this stage's scales are no longer needed
 
@@ -395,36 +434,35 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         // as one 16-byte store.
         const bool have_y = p.y != nullptr;
 #pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4)
+        for (int c = 0; c < 8; ++c)
 #pragma unroll
-          for (int lh = 0; lh < 2; ++lh)
+          for (int v = 0; v < 2; ++v) {
+            const int h = c >> 2, j4 = (c >> 1) & 1, lh = c & 1;
+            uint32_t hb[4];
 #pragma unroll
-            for (int v = 0; v < 2; ++v) {
-              uint32_t hb[4];
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const float2 val = acc[(j4 * 2 + lh) * 8 + 2 * k + v];
-                hb[k] = pack_half2_rn(val.x, val.y);
-              }
-              // round r: send block t0^r to lane t0^r, receive my block t0 from it
-              uint32_t o0 = hb[0], o1 = hb[1], o2 = hb[2], o3 = hb[3];
-#pragma unroll
-              for (int r = 1; r < 4; ++r) {
-                const int idx = t0 ^ r;
-                const uint32_t send =
-                    idx == 0 ? hb[0] : (idx == 1 ? hb[1] : (idx == 2 ? hb[2] : hb[3]));
-                const uint32_t got = __shfl_xor_sync(0xffffffffu, send, r);
-                o0 = idx == 0 ? got : o0;
-                o1 = idx == 1 ? got : o1;
-                o2 = idx == 2 ? got : o2;
-                o3 = idx == 3 ? got : o3;
-              }
-              const int row = w.m0 + BM * rank + 32 * q + 16 * lh + i0 + 8 * v;
-              const int col = w.n0 + h * 128 + 32 * j4 + 8 * t0;
-              const bool ok = have_y && row < p.M && col < p.N;
-              st_global_v4_if(p.y + static_cast<int64_t>(ok ? row : 0) * p.N + (ok ? col : 0),
-                              o0, o1, o2, o3, ok);
+            for (int k = 0; k < 4; ++k) {
+              const float2 val = acc[c * 8 + 2 * k + v];
+              hb[k] = pack_half2_rn(val.x, val.y);
             }
+            // round r: send block t0^r to lane t0^r, receive my block t0 from it
+            uint32_t o0 = hb[0], o1 = hb[1], o2 = hb[2], o3 = hb[3];
+#pragma unroll
+            for (int r = 1; r < 4; ++r) {
+              const int idx = t0 ^ r;
+              const uint32_t send =
+                  idx == 0 ? hb[0] : (idx == 1 ? hb[1] : (idx == 2 ? hb[2] : hb[3]));
+              const uint32_t got = __shfl_xor_sync(0xffffffffu, send, r);
+              o0 = idx == 0 ? got : o0;
+              o1 = idx == 1 ? got : o1;
+              o2 = idx == 2 ? got : o2;
+              o3 = idx == 3 ? got : o3;
+            }
+            const int row = w.m0 + BM * rank + 32 * q + 16 * lh + i0 + 8 * v;
+            const int col = w.n0 + tile_col(h * 128 + hh * 64 + 32 * j4 + 8 * t0);
+            const bool oky = have_y && row < p.M && col < p.N;
+            st_global_v4_if(p.y + static_cast<int64_t>(oky ? row : 0) * p.N + (oky ? col : 0),
+                            o0, o1, o2, o3, oky);
+          }
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
       }
@@ -472,55 +510,42 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       if (lane == 0 && rank == 0) {
         // ============================================================ MMA issuer (leader)
         int64_t last_mma = -1;
-        for (int64_t it = 0; it < iters; ++it) {
+        bool ok = true;
+        for (int64_t it = 0; ok && it < iters; ++it) {
           const int s = static_cast<int>(it % kStages), b = static_cast<int>(it & 1);
           const uint32_t ph = static_cast<uint32_t>((it / kStages) & 1);
           if (!mbar_wait(&lfull[s], ph, abort_flag) ||
-              !mbar_wait_cluster(&mfull[s], ph, abort_flag) ||
-              !mbar_wait_cluster(&tempty[b], static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
-                                 abort_flag)) {
-            fail();
+              !mbar_wait_cluster(&mfull[s], ph, abort_flag)) {
+            ok = false;
             break;
           }
-          tc_fence_after_sync();
           const uint32_t a_addr = smem_addr(stages + s * kStageBytes);
           const uint64_t adesc = smem_desc_k_sw128(a_addr);
-          const uint64_t bdesc = smem_desc_k_sw128(a_addr + kABytes);
-          const uint32_t d = tbase + b * BN;
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait_cluster(&tempty[2 * b + h], static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
+                                   abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after_sync();
+            // half h: W rows [64h, 64h+64) of each CTA's tile
+            const uint64_t bdesc = smem_desc_k_sw128(a_addr + kABytes + h * 64 * 128);
+            const uint32_t d = tbase + b * BN + h * kHalfN;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
+            for (int k = 0; k < 4; ++k)
+              mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
+            tc_commit_pair_multicast(&tfull[2 * b + h], 0x3);
+          }
+          if (!ok) break;
           tc_commit_pair_multicast(&empty[s], 0x3);
-          tc_commit_pair_multicast(&tfull[b], 0x3);
           last_mma = it;
         }
+        if (!ok) fail();
         // nothing may still write TMEM when it is released
         if (last_mma >= 0)
-          (void)mbar_wait(&tfull[last_mma & 1], static_cast<uint32_t>((last_mma >> 1) & 1),
-                          nullptr);
-      } else if (lane == 0) {
-        // ============================================================ relay (peer)
-        // One cross-SM arrival per event: "this CTA's operands of group it are
-        // unpacked" and "this CTA's accumulator of group it-1 is drained".
-        for (int64_t it = 0; it <= iters; ++it) {
-          if (it < iters) {
-            const int s = static_cast<int>(it % kStages);
-            if (!mbar_wait(&lfull[s], static_cast<uint32_t>((it / kStages) & 1), abort_flag)) {
-              fail();
-              break;
-            }
-            mbar_arrive_cluster(cluster_map(&mfull[s], 0));
-          }
-          if (it >= 1) {
-            const int64_t j = it - 1;
-            const int b = static_cast<int>(j & 1);
-            if (!mbar_wait(&tempty[b], static_cast<uint32_t>((j >> 1) & 1), abort_flag)) {
-              fail();
-              break;
-            }
-            mbar_arrive_cluster(cluster_map(&tempty[b], 0));
-          }
-        }
+          (void)mbar_wait(&tfull[2 * (last_mma & 1) + 1],
+                          static_cast<uint32_t>((last_mma >> 1) & 1), nullptr);
       }
     } else {
       // ============================================================== unpackers
@@ -528,11 +553,13 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       TileWalk w;
       w.start(p);
       float sa_d = (!p.sa_by_tma && iters > 0) ? sa_direct_load(p, w, rank, lt) : 0.f;
+      const uint32_t mfull_leader = cluster_map(&mfull[0], 0);
       for (int64_t it = 0; it < iters; ++it) {
         const int s = static_cast<int>(it % kStages);
         TileWalk wn = w;
         wn.next(p);
-        if (!mbar_wait(&pfull[s], static_cast<uint32_t>((it / kStages) & 1), abort_flag)) {
+        const bool ok = mbar_wait(&pfull[s], static_cast<uint32_t>((it / kStages) & 1), abort_flag);
+        if (named_bar_any(kBarUnpack, kUnpackThreads, !ok)) {
           fail();
           break;
         }
@@ -540,8 +567,11 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         unpack_stage(p, w, lt, stage, sa_d);
         if (!p.sa_by_tma && it + 1 < iters) sa_d = sa_direct_load(p, wn, rank, lt);
         fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&lfull[s]);
+        named_bar_sync(kBarUnpack, kUnpackThreads);
+        if (lt == 0) {
+          mbar_arrive(&lfull[s]);
+          if (rank == 1) mbar_arrive_cluster(mfull_leader + 8u * s);
+        }
         w = wn;
       }
     }
