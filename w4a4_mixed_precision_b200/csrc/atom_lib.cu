@@ -13,7 +13,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int64_t kMaxK = 32768;  // the permutation is staged as uint16 in shared memory
+constexpr int64_t kMaxK = atomk::kQuantMaxK;  // gather offsets are uint16 in shared memory
 
 struct DeviceState {
   bool probed = false;
@@ -23,6 +23,8 @@ struct DeviceState {
   bool gemm_attr[2] = {false, false};
   int gemm_clusters[2] = {0, 0};  // co-resident CTA pairs of the GEMM kernel
   uint32_t quant_smem_set = 0;
+  uint32_t quant_occ_smem = 0;  // shared-memory size the cached occupancy is for
+  int quant_occ = 0;            // co-resident quantizer CTAs per SM at that size
 };
 
 DeviceState g_devices[kMaxDevices];
@@ -92,10 +94,18 @@ atom_status_t launch_quant(const void *x, int64_t rows, int64_t K, int64_t ld,
       return ATOM_ERR_CUDA;
     dev->quant_smem_set = L.total;
   }
-  // CTAs per SM: limited by 2048 threads and ~228 KB of shared memory (1 KB reserved per CTA).
-  int per_sm = static_cast<int>((228u * 1024u) / (L.total + 1024u));
-  per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
-  const int64_t want = static_cast<int64_t>(per_sm) * dev->sm_count;
+  // One persistent wave: as many CTAs as fit on the device at once.
+  if (dev->quant_occ_smem != L.total) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, atomk::reorder_quant_kernel,
+                                                      atomk::kQuantThreads,
+                                                      L.total) != cudaSuccess)
+      return ATOM_ERR_CUDA;
+    dev->quant_occ = per_sm < 1 ? 1 : per_sm;
+    dev->quant_occ_smem = L.total;
+  }
+  const int64_t want = static_cast<int64_t>(dev->quant_occ) * dev->sm_count;
   const int grid = static_cast<int>(rows < want ? rows : want);
   atomk::reorder_quant_kernel<<<grid, atomk::kQuantThreads, L.total,
                                 reinterpret_cast<cudaStream_t>(stream)>>>(

@@ -7,20 +7,29 @@
 // (fields "Weight group size" = 128 and "notes": every contiguous run of 128
 // elements is one group quantized independently; 128 high-precision channels).
 //
-// Design (memory-bound, so the goal is to keep HBM busy):
+// Design (HBM-bound, so the aim is to keep HBM busy with few instructions per
+// element):
 //  * each CTA is persistent over rows r = blockIdx.x + i*gridDim.x; a whole
 //    fp16 row is brought into shared memory by one bulk copy (TMA engine,
-//    mbarrier completion), S rows in flight per CTA;
-//  * the permutation is built once per CTA in shared memory (uint16 [K]) while
-//    the first rows are in flight: a bitmap of the outlier channels, a block
-//    scan of the non-outlier counts, then the outlier list at the tail;
-//  * 8 lanes quantize one group (16 reordered elements per lane), 4 groups per
-//    warp per pass: gather from the staged row through the permutation,
-//    shuffle-reduce amax over the 8 lanes, one IEEE division each for scale and
-//    inv, codes by round-half-even via the 1.5*2^23 add (exact for |t| < 2^22),
-//    nibble packing in registers, 8-byte (INT4) or 16-byte (INT8) stores;
-//  * the gather order inside a lane is rotated per lane so that the 32 lanes of
-//    a warp read 32 distinct shared-memory banks.
+//    mbarrier completion), up to kQuantMaxStages rows in flight per CTA; each
+//    warp frees a stage through its own arrival on an "empty" mbarrier, so the
+//    warps of a CTA never wait for one another while the ring has room;
+//  * at start-up each CTA turns the outlier list into a gather table in shared
+//    memory (uint16 [K]): for every group and lane, the byte offsets inside a
+//    staged row of the 16 channels that lane quantizes, in the lane's gather
+//    order. Reordered position p holds the p-th non-outlier channel for
+//    p < K-128 and outlier_idx[p-(K-128)] after that (bitmap of the outliers,
+//    block scan of the non-outlier counts);
+//  * 8 lanes quantize one group (16 elements per lane), 4 groups per warp per
+//    pass: two conflict-free 16-byte table loads, 16 gathered halves, amax by
+//    shuffles over the 8 lanes, one IEEE division each for scale and inv, code
+//    bits from the low byte of fp32(1.5*2^23 + x*inv) (round half to even,
+//    exact for |t| < 2^22), byte permutes to
+//    pack, one 8-byte (INT4) or 16-byte (INT8) store per lane;
+//  * a dense-group lane gathers its 16 elements rotated by an even amount that
+//    depends on its position, so the 32 lanes of a warp read 32 distinct
+//    shared-memory banks; the packed 8 bytes are rotated back with two byte
+//    permutes.
 #pragma once
 
 #include "ptx.cuh"
@@ -28,11 +37,14 @@
 namespace atomk {
 
 constexpr int kQuantThreads = 256;
+constexpr int kQuantWarps = kQuantThreads / 32;
 constexpr int kQuantMaxStages = 4;
+// Gather-table entries are 16-bit byte offsets into a staged fp16 row.
+constexpr int kQuantMaxK = 32768;
 
 struct QuantLayout {
   // Byte offsets inside dynamic shared memory.
-  uint32_t bitmap, perm, stages, total;
+  uint32_t bitmap, table, stages, total;
   uint32_t row_bytes;
   int stages_n;
 };
@@ -41,11 +53,32 @@ __host__ __device__ inline QuantLayout quant_layout(int K, int stages_n) {
   QuantLayout L;
   L.row_bytes = 2u * static_cast<uint32_t>(K);
   L.bitmap = 256;                                                  // after barriers and flags
-  L.perm = L.bitmap + ((static_cast<uint32_t>(K) / 8u + 15u) & ~15u);
-  L.stages = (L.perm + L.row_bytes + 127u) & ~127u;
+  L.table = L.bitmap + ((static_cast<uint32_t>(K) / 8u + 15u) & ~15u);
+  L.stages = (L.table + L.row_bytes + 127u) & ~127u;
   L.stages_n = stages_n;
   L.total = L.stages + static_cast<uint32_t>(stages_n) * L.row_bytes;
   return L;
+}
+
+// Gather rotation of lane `sub` (0..7) in team `team` (0..3) for a dense group.
+__device__ __forceinline__ int quant_rotation(int sub, int team) {
+  return 2 * ((sub >> 2) & 1) + 4 * team;
+}
+
+// Table slot of reordered position p: group g = p/128 is quantized by team
+// g%4 of some warp; lane sub = (p%128)/16 takes element e = p%16 at gather step
+// (e - rot) mod 16. Slots 0..7 of all 8 lanes come first, then slots 8..15, so
+// that each 8-lane team reads 128 contiguous bytes per 16-byte table load.
+__device__ __forceinline__ int quant_table_index(int p, int Gd) {
+  const int g = p >> 7, sub = (p >> 4) & 7, e = p & 15;
+  const int rot = g < Gd ? quant_rotation(sub, g & 3) : 0;
+  const int slot = (e - rot) & 15;
+  return (((g * 2 + (slot >> 3)) * 8 + sub) << 3) + (slot & 7);
+}
+
+// Low bytes of four 32-bit words, in order, as one word.
+__device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
 __global__ void __launch_bounds__(kQuantThreads)
@@ -54,11 +87,12 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
                      int8_t *__restrict__ q8, float *__restrict__ scales, int stages_n) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const QuantLayout L = quant_layout(K, stages_n);
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem);             // [kQuantMaxStages]
-  volatile int *flags = reinterpret_cast<volatile int *>(smem + 64);  // [0] bad list
-  int *warp_sums = reinterpret_cast<int *>(smem + 128);            // [8]
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem);                 // [kQuantMaxStages]
+  uint64_t *empty = full + kQuantMaxStages;                            // [kQuantMaxStages]
+  volatile int *flags = reinterpret_cast<volatile int *>(smem + 96);  // [0] bad list, [1] abort
+  int *warp_sums = reinterpret_cast<int *>(smem + 128);               // [8]
   uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem + L.bitmap);
-  uint16_t *perm = reinterpret_cast<uint16_t *>(smem + L.perm);
+  uint16_t *table = reinterpret_cast<uint16_t *>(smem + L.table);
   uint8_t *stage_base = smem + L.stages;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -67,14 +101,18 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
   const int64_t grid = gridDim.x;
 
   if (tid == 0) {
-    for (int s = 0; s < stages_n; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < stages_n; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kQuantWarps);
+    }
     flags[0] = 0;
+    flags[1] = 0;
     fence_mbar_init();
   }
   for (int w = tid; w < K / 32; w += kQuantThreads) bitmap[w] = 0u;
   __syncthreads();
 
-  // Put the first rows in flight before building the permutation.
+  // Put the first rows in flight before building the table.
   if (tid == 0) {
     for (int s = 0; s < stages_n; ++s) {
       const int64_t r = blockIdx.x + s * grid;
@@ -85,7 +123,7 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     }
   }
 
-  // ---- permutation: ascending non-outlier channels, then the outlier list.
+  // ---- gather table: ascending non-outlier channels, then the outlier list.
   if (tid < 128) {
     const int c = outlier_idx[tid];
     if (c < 0 || c >= K) {
@@ -117,13 +155,13 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     while (bits) {
       const int b = __ffs(bits) - 1;
       bits &= bits - 1;
-      if (pos < Kd) perm[pos] = static_cast<uint16_t>(w * 32 + b);
+      if (pos < Kd) table[quant_table_index(pos, Gd)] = static_cast<uint16_t>(2 * (w * 32 + b));
       ++pos;
     }
   }
   if (tid < 128) {
     const int c = outlier_idx[tid];
-    if (c >= 0 && c < K) perm[Kd + tid] = static_cast<uint16_t>(c);
+    if (c >= 0 && c < K) table[quant_table_index(Kd + tid, Gd)] = static_cast<uint16_t>(2 * c);
   }
   __syncthreads();
 
@@ -137,39 +175,49 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     return;
   }
 
-  // ---- per-lane work assignment (fixed for the whole kernel)
-  const int sub = lane & 7;        // lane within its 8-lane group team
-  const int team = lane >> 3;      // which of the warp's 4 groups
-  const int rot_dense = 2 * ((sub >> 2) & 1) + 4 * team;  // even, 0..14
+  // ---- per-lane constants: group g = pass*32 + 4*warp + team, elements
+  // [16*sub, 16*sub + 16) of the group.
+  const int sub = lane & 7;
+  const int team = lane >> 3;
   const unsigned team_mask = 0xFFu << (8 * team);
+  // Byte permutes that rotate the packed dense 8 bytes left by rot/2 bytes.
+  const int krot = quant_rotation(sub, team) >> 1;
+  uint32_t sel_lo = 0, sel_hi = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    sel_lo |= static_cast<uint32_t>((j - krot) & 7) << (4 * j);
+    sel_hi |= static_cast<uint32_t>((j + 4 - krot) & 7) << (4 * j);
+  }
 
-  int64_t aborted_at = -1;
+  int64_t done = 0;  // rows this CTA has finished
   for (int64_t i = 0;; ++i) {
     const int64_t r = blockIdx.x + i * grid;
     if (r >= rows) break;
     const int s = static_cast<int>(i % stages_n);
-    const uint32_t parity = static_cast<uint32_t>((i / stages_n) & 1);
-    const bool ok = mbar_wait(&full[s], parity, nullptr);
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) report_status(6 /* ATOM_ERR_TIMEOUT */);
-      aborted_at = i;
+    if (!mbar_wait(&full[s], static_cast<uint32_t>((i / stages_n) & 1), &flags[1])) {
+      if (lane == 0) {
+        report_status(6 /* ATOM_ERR_TIMEOUT */);
+        flags[1] = 1;
+      }
       break;
     }
-    const __half *row = reinterpret_cast<const __half *>(stage_base + s * L.row_bytes);
+    const uint8_t *row = stage_base + s * L.row_bytes;
 
     for (int gb = 0; gb < G; gb += 32) {
       const int g = gb + warp * 4 + team;
       if (g > Gd) continue;  // whole 8-lane teams skip together
       const bool dense = g < Gd;
-      const int rot = dense ? rot_dense : 0;
-      const int j0 = g * 128 + sub * 16;
-      float v[16];
+      const uint16_t *tb = table + ((g * 2) * 8 + sub) * 8;
+      const uint4 oa = *reinterpret_cast<const uint4 *>(tb);       // slots 0..7
+      const uint4 ob = *reinterpret_cast<const uint4 *>(tb + 64);  // slots 8..15
+      const uint32_t offs[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
+      float2 v[8];
       float amax = 0.f;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int c = perm[j0 + ((e + rot) & 15)];
-        v[e] = __half2float(row[c]);
-        amax = fmaxf(amax, fabsf(v[e]));
+      for (int j = 0; j < 8; ++j) {
+        v[j].x = __half2float(*reinterpret_cast<const __half *>(row + (offs[j] & 0xFFFFu)));
+        v[j].y = __half2float(*reinterpret_cast<const __half *>(row + (offs[j] >> 16)));
+        amax = fmaxf(amax, fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
       }
       amax = fmaxf(amax, __shfl_xor_sync(team_mask, amax, 4));
       amax = fmaxf(amax, __shfl_xor_sync(team_mask, amax, 2));
@@ -180,57 +228,64 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
         scale = __fdiv_rn(amax, qmax);
         inv = __fdiv_rn(qmax, amax);
       }
-      // code bits: low bits of fp32(1.5*2^23 + rint(x*inv)) are the two's complement code
-      uint32_t bits[16];
+      // code bits: the low byte of fp32(1.5*2^23 + rint(x*inv)) is the two's complement code
+      // __fmul_rn/__fadd_rn are never contracted into an FMA: the product must
+      // be rounded to fp32 before the 1.5*2^23 add rounds it to an integer.
+      uint32_t b[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e)
-        bits[e] = __float_as_uint(__fadd_rn(__fmul_rn(v[e], inv), 12582912.f));
+      for (int j = 0; j < 8; ++j) {
+        b[2 * j] = __float_as_uint(__fadd_rn(__fmul_rn(v[j].x, inv), 12582912.f));
+        b[2 * j + 1] = __float_as_uint(__fadd_rn(__fmul_rn(v[j].y, inv), 12582912.f));
+      }
       if (dense) {
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          lo |= (bits[e] & 0xFu) << (4 * e);
-          hi |= (bits[e + 8] & 0xFu) << (4 * e);
-        }
-        // slot e holds element (e + rot) mod 16: rotate the 64-bit word left by 4*rot
-        uint64_t p = (static_cast<uint64_t>(hi) << 32) | lo;
-        const int sh = 4 * rot;
-        if (sh) p = (p << sh) | (p >> (64 - sh));
+        // gather slot e holds element (e + rot) mod 16 of the lane's 16
+        const uint32_t ev0 = low_bytes4(b[0], b[2], b[4], b[6]);
+        const uint32_t od0 = low_bytes4(b[1], b[3], b[5], b[7]);
+        const uint32_t ev1 = low_bytes4(b[8], b[10], b[12], b[14]);
+        const uint32_t od1 = low_bytes4(b[9], b[11], b[13], b[15]);
+        const uint32_t lo = (ev0 & 0x0F0F0F0Fu) | ((od0 << 4) & 0xF0F0F0F0u);
+        const uint32_t hi = (ev1 & 0x0F0F0F0Fu) | ((od1 << 4) & 0xF0F0F0F0u);
         *reinterpret_cast<uint2 *>(q4 + r * q4_row + g * 64 + sub * 8) =
-            make_uint2(static_cast<uint32_t>(p), static_cast<uint32_t>(p >> 32));
+            make_uint2(__byte_perm(lo, hi, sel_lo), __byte_perm(lo, hi, sel_hi));
       } else {
         uint4 o;
-        o.x = (bits[0] & 0xFFu) | ((bits[1] & 0xFFu) << 8) | ((bits[2] & 0xFFu) << 16) |
-              ((bits[3] & 0xFFu) << 24);
-        o.y = (bits[4] & 0xFFu) | ((bits[5] & 0xFFu) << 8) | ((bits[6] & 0xFFu) << 16) |
-              ((bits[7] & 0xFFu) << 24);
-        o.z = (bits[8] & 0xFFu) | ((bits[9] & 0xFFu) << 8) | ((bits[10] & 0xFFu) << 16) |
-              ((bits[11] & 0xFFu) << 24);
-        o.w = (bits[12] & 0xFFu) | ((bits[13] & 0xFFu) << 8) | ((bits[14] & 0xFFu) << 16) |
-              ((bits[15] & 0xFFu) << 24);
+        o.x = low_bytes4(b[0], b[1], b[2], b[3]);
+        o.y = low_bytes4(b[4], b[5], b[6], b[7]);
+        o.z = low_bytes4(b[8], b[9], b[10], b[11]);
+        o.w = low_bytes4(b[12], b[13], b[14], b[15]);
         *reinterpret_cast<uint4 *>(q8 + r * 128 + sub * 16) = o;
       }
       if (sub == 0) scales[static_cast<int64_t>(g) * rows + r] = scale;
     }
 
-    __syncthreads();  // every warp is done with this stage
-    if (tid == 0) {
-      const int64_t nr = r + stages_n * grid;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    done = i + 1;
+
+    // Refill the stage of the previous row: one row of slack, so the issuing
+    // thread rarely waits for the slowest warp.
+    if (tid == 0 && i >= 1) {
+      const int64_t j = i - 1;
+      const int64_t nr = blockIdx.x + (j + stages_n) * grid;
       if (nr < rows) {
-        mbar_arrive_expect_tx(&full[s], L.row_bytes);
-        bulk_load(stage_base + s * L.row_bytes, x + nr * ld, L.row_bytes, &full[s]);
+        const int sj = static_cast<int>(j % stages_n);
+        if (!mbar_wait(&empty[sj], static_cast<uint32_t>((j / stages_n) & 1), &flags[1])) {
+          report_status(6 /* ATOM_ERR_TIMEOUT */);
+          flags[1] = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[sj], L.row_bytes);
+        bulk_load(stage_base + sj * L.row_bytes, x + nr * ld, L.row_bytes, &full[sj]);
       }
     }
   }
 
-  // After a timeout, give the copies still in flight a bounded chance to land
+  // After an abort, give the copies still in flight a bounded chance to land
   // before the CTA's shared memory is released.
-  if (aborted_at >= 0 && tid == 0) {
-    for (int k = 0; k < stages_n; ++k) {
-      const int64_t it = aborted_at + k;
-      if (blockIdx.x + it * grid < rows)
-        (void)mbar_wait(&full[it % stages_n], static_cast<uint32_t>((it / stages_n) & 1), nullptr);
-    }
+  if (tid == 0 && flags[1]) {
+    for (int64_t j = done; j < done + stages_n; ++j)
+      if (blockIdx.x + j * grid < rows)
+        (void)mbar_wait(&full[j % stages_n], static_cast<uint32_t>((j / stages_n) & 1), nullptr);
   }
 }
 
