@@ -19,36 +19,48 @@
 // M=256, N=128, K=32); half h takes W rows [64h, 64h+64) from each CTA, so
 // accumulator column j of half h is tile column 64h + (j mod 64) + 128*(j/64).
 // Two groups in flight x two halves gives four 128-column accumulators per
-// CTA, and the drain hands each half back as soon as it has read it, so the
-// tensor cores never wait for a whole group to be drained. The pairs are
-// persistent over tiles (m fastest). Roles in each CTA:
+// CTA, and the drain hands each half back as soon as it has read it. The pairs
+// are persistent over tiles (m fastest).
 //
-//   producer (warp 0, lane 0)  TMA copies of the group's packed INT4 tiles
-//                      (128 rows x 64 bytes of A and of W), or of the INT8
-//                      outlier tiles straight into MMA layout, plus the
-//                      group's sa and sw vectors, into a free stage.
+// Three shared-memory rings decouple the stages, so that no stage holds a
+// buffer longer than its own step needs:
+//   packed ring   (TMA -> unpackers): one slot per INT4 group (128 rows x 64 B
+//                 of A and of W, plus the group's sw and sa vectors); the INT8
+//                 outlier group takes two slots (A8, then W8, each 128 x 128 B
+//                 in the 128-byte-swizzled MMA layout). Freed by the unpackers.
+//   operand ring  (unpackers -> MMA): the group's K-major, 128-byte-swizzled
+//                 int8 A and W tiles. Freed by the MMA's commit.
+//   scale ring    (unpackers -> drain): sa and sw laid out for the drain's
+//                 TMEM fragments. Freed by the drain.
+// Roles in each CTA:
+//
+//   producer (warp 0, lane 0)  TMA copies into the packed ring.
 //   warp 1, lane 0     (leader CTA) per group and half: 4 x 2-SM MMA into a
 //                      128-column TMEM accumulator, commit to both CTAs' "half
 //                      full" barrier; after both halves commit to both CTAs'
-//                      "stage empty" barrier.
-//   unpack warps 2..7  expand each nibble of the staged packed tiles to a byte
+//                      "operands free" barrier.
+//   unpack warps 2..7  expand each nibble of the packed tiles to a byte
 //                      holding 16*q (x << 4 & 0xF0 / x & 0xF0), store K-major
-//                      with the 128-byte swizzle, and lay the scales out for
-//                      the drain; then one thread signals "operands ready"
-//                      locally and, in the peer CTA, to the leader.
-//   drain warps 8..15  read the partials with the 16x256b TMEM shape (a thread
-//                      holds 4 rows x 2 columns of every 8-column block), release
-//                      each half once read (one arrival per CTA, on the leader),
-//                      and accumulate sa*sw*P into fp32 registers. After the
+//                      with the 128-byte swizzle (the INT8 group is copied),
+//                      and lay the scales out for the drain; then one thread
+//                      signals "operands ready" locally and, from the peer CTA,
+//                      to the leader.
+//   drain warps 8..15  warps 8..11 drain accumulator half 0 and 12..15 half 1:
+//                      each thread reads one TMEM lane (one output row) with
+//                      the 32x32b shape, 16 columns per load, accumulates
+//                      sa*sw*P into 128 fp32 registers, and each half is
+//                      handed back to the MMA as soon as its four warps have
+//                      read it (one arrival per CTA, on the leader). After the
 //                      last group of a tile: fp16 stores.
 //
-// Exact integer -> float: F = float with the bits P + 0x4B400000 equals
-// 1.5*2^23 + P exactly for |P| < 2^22 (one integer add per element; the
-// alternative of pre-filling TMEM with that bias doubles the TMEM traffic).
-// Dequantisation: with sw' = sw truncated to 22 significant bits, C*sw' is
-// exact for C = 1.5*2^23, so t = fma(F, sw', -C*sw') = round(P*sw') in one
-// instruction, then acc = fma(t, sa, acc); both run as packed f32x2 pairs.
-// (The truncation changes sw by less than 2^-21 relative.)
+// Exact integer -> float: F = float with the low 23 bits of P + 2^22 under the
+// exponent of 2^23 equals 1.5*2^23 + P exactly for |P| < 2^22 (one LOP3 per
+// element on the integer pipe; the alternative of pre-filling TMEM with that
+// bias doubles the TMEM traffic).
+// Dequantisation: with sa' = sa truncated to 22 significant bits, C*sa' is
+// exact for C = 1.5*2^23, so t = fma(F, sa', -C*sa') = round(P*sa') in one
+// instruction, then acc = fma(t, sw, acc); both run as packed f32x2 pairs.
+// (The truncation changes sa by less than 2^-21 relative.)
 //
 // Nibbles are expanded as 16*q so no sign extension is needed: INT4 partials
 // come out as exactly 256*P, and 1/256 is folded into sa. Both operands use
@@ -66,32 +78,42 @@ constexpr int BM = 128;          // A rows per CTA (256 per pair)
 constexpr int BN = 256;          // output columns per pair tile
 constexpr int BW = 128;          // W rows per CTA
 constexpr int kPairM = 2 * BM;
-constexpr int kStages = 4;
 constexpr int kThreads = 512;
 constexpr int kUnpackThreads = 192;  // warps 2..7
-// stage layout (bytes from a 1024-aligned stage base)
-constexpr uint32_t kABytes = BM * 128;                 // unpacked / INT8 A, 128-byte swizzle
-constexpr uint32_t kBBytes = BW * 128;                 // unpacked / INT8 W, 128-byte swizzle
-constexpr uint32_t kPackAOff = kABytes + kBBytes;      // packed A, 128 rows x 64 B
-constexpr uint32_t kPackWOff = kPackAOff + BM * 64;    // packed W, 128 rows x 64 B
-constexpr uint32_t kSwLinOff = kPackWOff + BW * 64;    // sw as copied (256 floats)
+constexpr int kUnpackWarps = kUnpackThreads / 32;
+constexpr int kNP = 6;           // packed ring slots
+constexpr int kNU = 3;           // operand ring slots
+constexpr int kNS = 6;           // scale ring slots
+// packed slot: INT4 A at 0, INT4 W at kPackWOff; or one INT8 tile at 0
+constexpr uint32_t kPackWOff = BM * 64;
+constexpr uint32_t kSwLinOff = 16384;                  // sw as copied (256 floats)
 constexpr uint32_t kSaLinOff = kSwLinOff + BN * 4;     // sa as copied (128 floats)
-constexpr uint32_t kSwOff = kSaLinOff + BM * 4;        // sw in drain order
-constexpr uint32_t kSaOff = kSwOff + BN * 4;           // sa in drain order
-constexpr uint32_t kStageBytes = 52u * 1024u;
+constexpr uint32_t kPSlot = 18u * 1024u;
+// operand slot: A then W, int8, K-major, 128-byte swizzle
+constexpr uint32_t kABytes = BM * 128;
+constexpr uint32_t kBBytes = BW * 128;
+constexpr uint32_t kUSlot = kABytes + kBBytes;
+// scale slot: sa then sw, in drain order
+constexpr uint32_t kSwOff = BM * 4;
+constexpr uint32_t kSSlot = (BM + BN) * 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBarBytes = 1024;
-constexpr uint32_t kSmemBytes = kBarBytes + kStages * kStageBytes + 1024;  // + alignment slack
-constexpr int kPackedChunks = (BM + BW) * 4;                                   // 16-B chunks / group
+constexpr uint32_t kUOff = kBarBytes;                    // from the 1024-aligned base
+constexpr uint32_t kPOff = kUOff + kNU * kUSlot;
+constexpr uint32_t kSOff = kPOff + kNP * kPSlot;
+constexpr uint32_t kSmemBytes = kSOff + kNS * kSSlot + 1024;  // + alignment slack
+constexpr int kPackedChunks = (BM + BW) * 4;                    // 16-B chunks per INT4 group
 constexpr int kChunksPerThread = (kPackedChunks + kUnpackThreads - 1) / kUnpackThreads;
+constexpr int kInt8Chunks = (kABytes + kBBytes) / 16;           // 16-B chunks of an INT8 group
 constexpr int kHalfN = BN / 2;   // columns per MMA / accumulator half
 constexpr uint32_t kIdesc = idesc_i8(kPairM, kHalfN);
-constexpr uint32_t kBias = 0x4B400000u;  // bits of 1.5 * 2^23
 constexpr float kBiasF = 12582912.0f;
-constexpr int kUnpackRegs = 56;
-constexpr int kDrainRegs = 200;
-static_assert(kSaOff + BM * 4 <= kStageBytes, "stage overflow");
-static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+constexpr int kUnpackRegs = 72;
+constexpr int kDrainRegs = 184;
+static_assert(kSaLinOff + BM * 4 <= kPSlot, "packed slot overflow");
+static_assert(kABytes <= kSwLinOff && kBBytes <= kSwLinOff, "INT8 tile must fit a packed slot");
+static_assert(kPSlot % 1024 == 0 && kUSlot % 1024 == 0, "slots must keep 1024-byte alignment");
+static_assert(kSOff % 16 == 0 && kSSlot % 16 == 0, "scale slots must be 16-byte aligned");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 static_assert(2 * 128 * (kUnpackRegs + kDrainRegs) == 65536, "register split must fill the file");
 }  // namespace gemm_cfg
@@ -156,6 +178,19 @@ struct TileWalk {
   }
 };
 
+// Position in a ring of n slots: slot index and the parity of the slot's
+// current use (flips each time the index wraps).
+struct RingPos {
+  int idx = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void next(int n) {
+    if (++idx == n) {
+      idx = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
 __device__ __forceinline__ int64_t pair_iterations(const GemmParams &p) {
   const int pair = static_cast<int>(blockIdx.x >> 1), pairs = static_cast<int>(gridDim.x >> 1);
   const int mine = p.tiles > pair ? (p.tiles - pair + pairs - 1) / pairs : 0;
@@ -171,60 +206,66 @@ __device__ __forceinline__ int tile_col(int c) {
   return ((j >> 6) << 7) + (h << 6) + (j & 63);
 }
 
-// Scale layouts in a stage, ordered for the drain's 16x256b fragments:
-//  sa: row r = 32q + i + 8k (i < 8, k < 4) at q*32 + i*4 + k, so a thread's four
-//      rows are one 16-byte load;
-//  sw: accumulator column c = 16S + 8u + 2t + e (t < 4, e, u < 2) at
-//      (4S + t)*4 + 2u + e, so a thread's four columns of a 16-column block are
-//      one 16-byte load. The stored value is sw of tile column tile_col(c),
-//      truncated to 22 significant bits.
-__device__ __forceinline__ int sa_slot(int r) { return (r >> 5) * 32 + (r & 7) * 4 + ((r >> 3) & 3); }
-__device__ __forceinline__ int sw_slot(int n) {
-  const int w = n & 15;
-  return ((n >> 4) * 4 + ((w & 7) >> 1)) * 4 + ((w >> 3) << 1) + (w & 1);
-}
-
-// Expands this thread's share of the staged packed tiles into the swizzled
-// MMA operands and lays out the scales. `sa_direct` is this thread's sa value
-// when sa does not come through TMA (rows not 16-byte aligned).
-__device__ __forceinline__ void unpack_stage(const GemmParams &p, const TileWalk &w, int lt,
-                                             uint8_t *stage, float sa_direct) {
+// Scale slot layout: sa by local row (128 floats), then sw by accumulator
+// column (256 floats: entry c holds sw of tile column tile_col(c)), so a drain
+// thread, which owns one row, reads its sa once and the sw of 16 consecutive
+// accumulator columns as four 16-byte broadcast loads.
+// One INT4 group: expands this thread's share of the packed tiles in `pk`
+// into the swizzled int8 operands in `op`.
+__device__ __forceinline__ void unpack_int4(int lt, const uint8_t *pk, uint8_t *op) {
   using namespace gemm_cfg;
-  if (w.g < p.G - 1) {
 #pragma unroll
-    for (int i = 0; i < kChunksPerThread; ++i) {
-      const int c = lt + kUnpackThreads * i;
-      if (c < kPackedChunks) {
-        const bool is_a = c < BM * 4;
-        const int cc = c & 3;
-        const int row = (is_a ? c : c - BM * 4) >> 2;
-        const uint4 v = *reinterpret_cast<const uint4 *>(
-            stage + (is_a ? kPackAOff : kPackWOff) + row * 64 + cc * 16);
-        uint8_t *dst = stage + (is_a ? 0u : kABytes) + row * 128;
-        const uint4 lo = make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
-                                    (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
-        const uint4 hi = make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
-                                    v.w & 0xF0F0F0F0u);
-        const int sw = row & 7;
-        *reinterpret_cast<uint4 *>(dst + (((2 * cc) ^ sw) << 4)) = lo;
-        *reinterpret_cast<uint4 *>(dst + (((2 * cc + 1) ^ sw) << 4)) = hi;
-      }
+  for (int i = 0; i < kChunksPerThread; ++i) {
+    const int c = lt + kUnpackThreads * i;
+    if (c < kPackedChunks) {
+      const bool is_a = c < BM * 4;
+      const int cc = c & 3;
+      const int row = (is_a ? c : c - BM * 4) >> 2;
+      const uint4 v =
+          *reinterpret_cast<const uint4 *>(pk + (is_a ? 0u : kPackWOff) + row * 64 + cc * 16);
+      uint8_t *dst = op + (is_a ? 0u : kABytes) + row * 128;
+      const uint4 lo = make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
+                                  (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
+      const uint4 hi = make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
+                                  v.w & 0xF0F0F0F0u);
+      const int sw = row & 7;
+      *reinterpret_cast<uint4 *>(dst + (((2 * cc) ^ sw) << 4)) = lo;
+      *reinterpret_cast<uint4 *>(dst + (((2 * cc + 1) ^ sw) << 4)) = hi;
     }
   }
+}
+
+// The INT8 outlier group: both tiles arrived already in the swizzled MMA
+// layout (A8 in `pk_a`, W8 in `pk_w`, both 1024-byte aligned like `op`), so
+// they are copied byte for byte.
+__device__ __forceinline__ void copy_int8(int lt, const uint8_t *pk_a, const uint8_t *pk_w,
+                                          uint8_t *op) {
+  using namespace gemm_cfg;
+  for (int c = lt; c < kInt8Chunks; c += kUnpackThreads) {
+    const bool is_a = c < static_cast<int>(kABytes / 16);
+    const uint32_t off = (is_a ? c : c - kABytes / 16) * 16u;
+    *reinterpret_cast<uint4 *>(op + (is_a ? 0u : kABytes) + off) =
+        *reinterpret_cast<const uint4 *>((is_a ? pk_a : pk_w) + off);
+  }
+}
+
+// Lays the group's scales out for the drain (threads 0..127: sa; 128..191: sw).
+// `sa_direct` is this thread's sa value when sa does not come through TMA.
+__device__ __forceinline__ void layout_scales(const GemmParams &p, int lt, const uint8_t *pk,
+                                              uint8_t *ss, float sa_direct) {
+  using namespace gemm_cfg;
   if (lt < BM) {
-    const float v = p.sa_by_tma ? reinterpret_cast<const float *>(stage + kSaLinOff)[lt] : sa_direct;
-    reinterpret_cast<float *>(stage + kSaOff)[sa_slot(lt)] = v;
+    reinterpret_cast<float *>(ss)[lt] =
+        p.sa_by_tma ? reinterpret_cast<const float *>(pk + kSaLinOff)[lt] : sa_direct;
   } else {
     constexpr int kSwThreads = kUnpackThreads - BM;   // threads laying out sw
     static_assert(kSwThreads > 0, "unpack threads must cover sa and sw");
 #pragma unroll
     for (int k = 0; k < (BN + kSwThreads - 1) / kSwThreads; ++k) {
       const int j = lt - BM + kSwThreads * k;
-      if (j < BN) {
-        const float v = reinterpret_cast<const float *>(stage + kSwLinOff)[tile_col(j)];
-        reinterpret_cast<float *>(stage + kSwOff)[sw_slot(j)] =
-            __uint_as_float(__float_as_uint(v) & 0xFFFFFFFCu);
-      }
+      if (j < BN)
+        reinterpret_cast<float *>(ss + kSwOff)[j] =
+            reinterpret_cast<const float *>(pk + kSwLinOff)[tile_col(j)];
     }
   }
 }
@@ -250,7 +291,6 @@ struct GemmMaps {
 };
 
 // Hardware barrier ids for the role-internal gathers (0 is __syncthreads).
-constexpr uint32_t kBarDrain = 1, kBarUnpack = 2;
 
 template <bool kPartials>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::kThreads, 1)
@@ -259,29 +299,41 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
 
-  uint64_t *pfull = reinterpret_cast<uint64_t *>(smem);  // [kStages] TMA -> unpackers
-  uint64_t *lfull = pfull + kStages;   // [kStages] unpacked (local) -> drain, MMA
-  uint64_t *mfull = lfull + kStages;   // [kStages] leader only: the peer's "unpacked"
-  uint64_t *empty = mfull + kStages;   // [kStages] MMA commit + local drain -> producer
-  uint64_t *tfull = empty + kStages;   // [4]       accumulator (buffer b, half h) at 2b+h
-  uint64_t *tempty = tfull + 4;        // [4]       leader only: both CTAs drained (b, h)
+  uint64_t *pfull = reinterpret_cast<uint64_t *>(smem);  // [kNP] TMA -> unpackers
+  uint64_t *pempty = pfull + kNP;      // [kNP] unpackers -> producer
+  uint64_t *ufull = pempty + kNP;      // [kNU] operands ready (local) -> MMA
+  uint64_t *mfull = ufull + kNU;       // [kNU] leader only: the peer's operands ready
+  uint64_t *uempty = mfull + kNU;      // [kNU] MMA commit -> unpackers (both CTAs)
+  uint64_t *sfull = uempty + kNU;      // [kNS] scales ready -> drain
+  uint64_t *sempty = sfull + kNS;      // [kNS] drain -> unpackers
+  uint64_t *tfull = sempty + kNS;      // [4]   accumulator (buffer b, half h) at 2b+h
+  uint64_t *tempty = tfull + 4;        // [4]   leader only: both CTAs drained (b, h)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 4);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  uint8_t *stages = smem + kBarBytes;
+  uint8_t *uring = smem + kUOff;
+  uint8_t *pring = smem + kPOff;
+  uint8_t *sring = smem + kSOff;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = static_cast<int>(cluster_cta_rank());
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kNP; ++s) {
       mbar_init(&pfull[s], 1);       // producer's expect_tx arrival (+ TMA bytes)
-      mbar_init(&lfull[s], 1);       // one unpack thread after the unpack gather
-      mbar_init(&mfull[s], 1);       // the peer's unpack thread
-      mbar_init(&empty[s], 1 + 8);   // MMA commit + local drain warps
+      mbar_init(&pempty[s], kUnpackWarps);   // lane 0 of each unpack warp
+    }
+    for (int s = 0; s < kNU; ++s) {
+      mbar_init(&ufull[s], kUnpackWarps);    // lane 0 of each local unpack warp
+      mbar_init(&mfull[s], kUnpackWarps);    // lane 0 of each of the peer's unpack warps
+      mbar_init(&uempty[s], 1);      // the MMA commit
+    }
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&sfull[s], kUnpackWarps);    // lane 0 of each unpack warp
+      mbar_init(&sempty[s], 8);      // one lane of each drain warp
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 2);      // one drain thread of each CTA
+      mbar_init(&tempty[i], 8);      // lane 0 of the half's 4 drain warps in each CTA
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -303,165 +355,112 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
 
   if (warp >= 8) {
     // ================================================================ drain
+    // Warp 8 + 4*hh + q owns TMEM lanes [32q, 32q+32) (the hardware's lane
+    // quarter for its warp) of accumulator half hh: thread `lane` holds row
+    // 32q + lane, columns [128hh, 128hh+128) of the accumulator, as 64 fp32
+    // pairs. The two halves are drained and released independently.
     regs_increase<kDrainRegs>();
     const int dw = warp - 8;
-    const int q = dw & 3;             // TMEM lane quarter this warp may access
-    const int hh = dw >> 2;           // which 64 columns of each accumulator half
-    const int t0 = lane & 3;          // column pair within an 8-column block
-    const int i0 = lane >> 2;         // row within a group of 8 lanes
+    const int q = dw & 3;
+    const int hh = dw >> 2;
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
-    const bool releaser = dw == 0 && lane == 0;
     const uint32_t tempty_leader = cluster_map(&tempty[0], 0);
+    const int lrow = 32 * q + lane;   // row within the CTA's 128
 
     float2 acc[64];
 #pragma unroll
     for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
-    const float2 negC = make_float2(-kBiasF, -kBiasF);
     TileWalk w;
     w.start(p);
-    bool aborted = false;
-    for (int64_t it = 0; it < iters && !aborted; ++it, w.next(p)) {
-      const int s = static_cast<int>(it % kStages), b = static_cast<int>(it & 1);
-      const uint32_t tph = static_cast<uint32_t>((it >> 1) & 1);
-      const bool ok = mbar_wait(&tfull[2 * b], tph, abort_flag) &&
-                      mbar_wait(&lfull[s], static_cast<uint32_t>((it / kStages) & 1), abort_flag);
-      if (named_bar_any(kBarDrain, 256, !ok)) {
-        fail();
+    RingPos sr;
+    for (int64_t it = 0; it < iters; ++it, w.next(p), sr.next(kNS)) {
+      const int b = static_cast<int>(it & 1), sl = sr.idx;
+      const bool ok =
+          mbar_wait_inline(&tfull[2 * b + hh], static_cast<uint32_t>((it >> 1) & 1), abort_flag) &&
+          mbar_wait_inline(&sfull[sl], sr.phase, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) fail();
         break;
       }
       tc_fence_after_sync();
-      const uint8_t *stage = stages + s * kStageBytes;
-      float4 sa4 = *reinterpret_cast<const float4 *>(stage + kSaOff + (q * 32 + i0 * 4) * 4);
-      if (w.g < p.G - 1) {  // INT4 partials are 256*P
-        sa4.x *= 0.00390625f;
-        sa4.y *= 0.00390625f;
-        sa4.z *= 0.00390625f;
-        sa4.w *= 0.00390625f;
-      }
-      const float *sw_s = reinterpret_cast<const float *>(stage + kSwOff);
-      const uint32_t tbuf = tbase + lane_base + b * BN + hh * 64;
+      const uint8_t *ss = sring + sl * kSSlot;
+      // t = fma(F, sa', -C*sa') = P*sa' exactly-rounded, with sa' = sa (times
+      // 1/256 for the INT4 groups, whose partials are 256*P) truncated to 22
+      // significant bits so that C*sa' is exact; then acc += t * sw.
+      float sa = reinterpret_cast<const float *>(ss)[lrow];
+      if (w.g < p.G - 1) sa *= 0.00390625f;
+      sa = __uint_as_float(__float_as_uint(sa) & 0xFFFFFFFCu);
+      const float2 sa2 = make_float2(sa, sa);
+      const float2 nc2 = make_float2(-kBiasF * sa, -kBiasF * sa);
+      const float4 *sw4 = reinterpret_cast<const float4 *>(ss + kSwOff) + hh * 32;
+      const uint32_t tcol = tbase + lane_base + b * BN + hh * kHalfN;
 
-      // chunk c = 4h + 2*j4 + lh: accumulator half h, 32 columns j4, TMEM lane half lh
       uint32_t ra[16], rb[16];
-      tmem_ld_16x256b_x4(tbuf, ra);
+      tmem_ld_x16(tcol, ra);
       tmem_ld_wait(ra);
-      float2 swk[4], nck[4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 8; ++c) {   // 16 accumulator columns per chunk
         uint32_t(&r)[16] = (c & 1) ? rb : ra;
         uint32_t(&rn)[16] = (c & 1) ? ra : rb;
-        const int h = c >> 2, j4 = (c >> 1) & 1, lh = c & 1;
-        const int c0 = h * 128 + hh * 64 + 32 * j4;   // accumulator column of this chunk
-        if (lh == 0) {
-          const float4 s4a = *reinterpret_cast<const float4 *>(sw_s + ((c0 >> 4) * 4 + t0) * 4);
-          const float4 s4b =
-              *reinterpret_cast<const float4 *>(sw_s + (((c0 >> 4) + 1) * 4 + t0) * 4);
-          swk[0] = make_float2(s4a.x, s4a.y);
-          swk[1] = make_float2(s4a.z, s4a.w);
-          swk[2] = make_float2(s4b.x, s4b.y);
-          swk[3] = make_float2(s4b.z, s4b.w);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) nck[k] = f2_mul(swk[k], negC);
-        }
-        if (c == 3 || c == 7) {
-          // every chunk of half h is in registers: hand the half back
-          tc_fence_before_sync();
-          bool ok2 = true;
-          if (c == 3) ok2 = mbar_wait(&tfull[2 * b + 1], tph, abort_flag);
-          if (named_bar_any(kBarDrain, 256, !ok2)) {
-            fail();
-            aborted = true;
-            break;
-          }
-          if (releaser) {
-            if (rank == 0)
-              mbar_arrive(&tempty[2 * b + h]);
-            else
-              mbar_arrive_cluster_relaxed(tempty_leader + 8u * (2 * b + h));
-          }
-          if (c == 3) tc_fence_after_sync();
-        }
-        if (c + 1 < 8) {
-          const int cn = c + 1;
-          tmem_ld_16x256b_x4(tbase + lane_base + (static_cast<uint32_t>(16 * (cn & 1)) << 16) +
-                                 b * BN + (cn >> 2) * 128 + hh * 64 + 32 * ((cn >> 1) & 1),
-                             rn);
-        }
+        if (c + 1 < 8) tmem_ld_x16(tcol + 16 * (c + 1), rn);
         if (kPartials) {
-          const int row0 = w.m0 + BM * rank + 32 * q + 16 * lh + i0;
-          const bool int4_group = w.g < p.G - 1;
+          // 16 consecutive tile columns; N % 8 == 0, so each 4-column store is
+          // wholly inside or wholly outside the matrix.
+          const int row = w.m0 + BM * rank + lrow;
+          const int col0 = w.n0 + tile_col(hh * kHalfN + 16 * c);
+          const int sh = w.g < p.G - 1 ? 8 : 0;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-#pragma unroll
-            for (int v = 0; v < 2; ++v) {
-              const int row = row0 + 8 * v;
-              const int col = w.n0 + tile_col(c0 + 8 * k + 2 * t0);
-              int32_t v0 = static_cast<int32_t>(r[4 * k + 2 * v]);
-              int32_t v1 = static_cast<int32_t>(r[4 * k + 2 * v + 1]);
-              if (int4_group) {
-                v0 >>= 8;
-                v1 >>= 8;
-              }
-              const bool okp = row < p.M && col < p.N;
-              st_global_v2_if(
-                  p.partials + (static_cast<int64_t>(w.g) * p.M + (okp ? row : 0)) * p.N +
-                      (okp ? col : 0),
-                  static_cast<uint32_t>(v0), static_cast<uint32_t>(v1), okp);
-            }
+          for (int v = 0; v < 4; ++v) {
+            const int col = col0 + 4 * v;
+            const bool okp = row < p.M && col < p.N;
+            int32_t *dst = p.partials +
+                           (static_cast<int64_t>(w.g) * p.M + (okp ? row : 0)) * p.N + (okp ? col : 0);
+            st_global_v4_if(dst, static_cast<uint32_t>(static_cast<int32_t>(r[4 * v]) >> sh),
+                            static_cast<uint32_t>(static_cast<int32_t>(r[4 * v + 1]) >> sh),
+                            static_cast<uint32_t>(static_cast<int32_t>(r[4 * v + 2]) >> sh),
+                            static_cast<uint32_t>(static_cast<int32_t>(r[4 * v + 3]) >> sh), okp);
+          }
         }
-        const float sa_lo = lh ? sa4.z : sa4.x, sa_hi = lh ? sa4.w : sa4.y;
-        float2 *a = acc + c * 8;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 flo = make_float2(__uint_as_float(r[4 * k] + kBias),
-                                         __uint_as_float(r[4 * k + 1] + kBias));
-          const float2 fhi = make_float2(__uint_as_float(r[4 * k + 2] + kBias),
-                                         __uint_as_float(r[4 * k + 3] + kBias));
-          a[2 * k] = f2_fma(f2_fma(flo, swk[k], nck[k]), make_float2(sa_lo, sa_lo), a[2 * k]);
-          a[2 * k + 1] =
-              f2_fma(f2_fma(fhi, swk[k], nck[k]), make_float2(sa_hi, sa_hi), a[2 * k + 1]);
+        for (int v = 0; v < 4; ++v) {
+          const float4 s4 = sw4[4 * c + v];
+          float2 *a = acc + 8 * c + 2 * v;
+          const float2 f0 = make_float2(__uint_as_float(biased_float_bits(r[4 * v])),
+                                        __uint_as_float(biased_float_bits(r[4 * v + 1])));
+          const float2 f1 = make_float2(__uint_as_float(biased_float_bits(r[4 * v + 2])),
+                                        __uint_as_float(biased_float_bits(r[4 * v + 3])));
+          a[0] = f2_fma(f2_fma(f0, sa2, nc2), make_float2(s4.x, s4.y), a[0]);
+          a[1] = f2_fma(f2_fma(f1, sa2, nc2), make_float2(s4.z, s4.w), a[1]);
         }
         if (c + 1 < 8) tmem_ld_wait(rn);
       }
-      if (aborted) break;
+      // this warp's lanes of the half are in registers: hand them back, and
+      // the group's scales with them
+      tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);  // this stage's scales are no longer needed
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(&tempty[2 * b + hh]);
+        else
+          mbar_arrive_cluster_relaxed(tempty_leader + 8u * (2 * b + hh));
+        mbar_arrive(&sempty[sl]);
+      }
 
       if (w.g == p.G - 1) {
-        // epilogue. For each 32-column chunk and row, the 4 lanes with the same
-        // i0 hold 2 columns of each of the 4 8-column blocks; a 4x4 transpose
-        // across those lanes gives lane t0 all 8 columns of block t0, written
-        // as one 16-byte store.
+        // epilogue: accumulator column 128hh + j is tile column
+        // 64hh + (j mod 64) + 128*(j/64): two runs of 64 columns per row.
+        const int row = w.m0 + BM * rank + lrow;
         const bool have_y = p.y != nullptr;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int seg = 0; seg < 2; ++seg)
 #pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const int h = c >> 2, j4 = (c >> 1) & 1, lh = c & 1;
-            uint32_t hb[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float2 val = acc[c * 8 + 2 * k + v];
-              hb[k] = pack_half2_rn(val.x, val.y);
-            }
-            // round r: send block t0^r to lane t0^r, receive my block t0 from it
-            uint32_t o0 = hb[0], o1 = hb[1], o2 = hb[2], o3 = hb[3];
-#pragma unroll
-            for (int r = 1; r < 4; ++r) {
-              const int idx = t0 ^ r;
-              const uint32_t send =
-                  idx == 0 ? hb[0] : (idx == 1 ? hb[1] : (idx == 2 ? hb[2] : hb[3]));
-              const uint32_t got = __shfl_xor_sync(0xffffffffu, send, r);
-              o0 = idx == 0 ? got : o0;
-              o1 = idx == 1 ? got : o1;
-              o2 = idx == 2 ? got : o2;
-              o3 = idx == 3 ? got : o3;
-            }
-            const int row = w.m0 + BM * rank + 32 * q + 16 * lh + i0 + 8 * v;
-            const int col = w.n0 + tile_col(h * 128 + hh * 64 + 32 * j4 + 8 * t0);
+          for (int v = 0; v < 8; ++v) {
+            const int col = w.n0 + 128 * seg + 64 * hh + 8 * v;
+            const float2 *a = acc + 32 * seg + 4 * v;
             const bool oky = have_y && row < p.M && col < p.N;
             st_global_v4_if(p.y + static_cast<int64_t>(oky ? row : 0) * p.N + (oky ? col : 0),
-                            o0, o1, o2, o3, oky);
+                            pack_half2_rn(a[0].x, a[0].y), pack_half2_rn(a[1].x, a[1].y),
+                            pack_half2_rn(a[2].x, a[2].y), pack_half2_rn(a[3].x, a[3].y), oky);
           }
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
@@ -474,57 +473,70 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       if (lane == 0) {
         TileWalk wp;
         wp.start(p);
-        int64_t produced = 0;
+        int64_t ls = 0;   // packed-ring load steps issued
+        RingPos pr;
         bool ok = true;
-        for (; produced < iters; ++produced, wp.next(p)) {
-          const int s = static_cast<int>(produced % kStages);
-          if (!mbar_wait(&empty[s], static_cast<uint32_t>(((produced / kStages) & 1) ^ 1),
-                         abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t *stage = stages + s * kStageBytes;
+        for (int64_t it = 0; ok && it < iters; ++it, wp.next(p)) {
           const int arow = wp.m0 + BM * rank, wrow = wp.n0 + BW * rank;
           const bool int4_group = wp.g < p.G - 1;
-          const uint32_t bytes = (int4_group ? (BM + BW) * 64u : kABytes + kBBytes) + BN * 4u +
-                                 (p.sa_by_tma ? BM * 4u : 0u);
-          mbar_arrive_expect_tx(&pfull[s], bytes);
-          if (int4_group) {
-            tma_load_2d(stage + kPackAOff, &maps.a4, wp.g * 64, arow, &pfull[s]);
-            tma_load_2d(stage + kPackWOff, &maps.w4, wp.g * 64, wrow, &pfull[s]);
-          } else {
-            tma_load_2d(stage, &maps.a8, 0, arow, &pfull[s]);
-            tma_load_2d(stage + kABytes, &maps.w8, 0, wrow, &pfull[s]);
+          for (int part = 0; part < (int4_group ? 1 : 2); ++part) {
+            const int s = pr.idx;
+            if (!mbar_wait(&pempty[s], pr.phase ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            uint8_t *slot = pring + s * kPSlot;
+            if (part == 0) {
+              const uint32_t bytes = (int4_group ? (BM + BW) * 64u : kABytes) + BN * 4u +
+                                     (p.sa_by_tma ? BM * 4u : 0u);
+              mbar_arrive_expect_tx(&pfull[s], bytes);
+              if (int4_group) {
+                tma_load_2d(slot, &maps.a4, wp.g * 64, arow, &pfull[s]);
+                tma_load_2d(slot + kPackWOff, &maps.w4, wp.g * 64, wrow, &pfull[s]);
+              } else {
+                tma_load_2d(slot, &maps.a8, 0, arow, &pfull[s]);
+              }
+              tma_load_2d(slot + kSwLinOff, &maps.sw, wp.n0, wp.g, &pfull[s]);
+              if (p.sa_by_tma) tma_load_2d(slot + kSaLinOff, &maps.sa, arow, wp.g, &pfull[s]);
+            } else {
+              mbar_arrive_expect_tx(&pfull[s], kBBytes);
+              tma_load_2d(slot, &maps.w8, 0, wrow, &pfull[s]);
+            }
+            ++ls;
+            pr.next(kNP);
           }
-          tma_load_2d(stage + kSwLinOff, &maps.sw, wp.n0, wp.g, &pfull[s]);
-          if (p.sa_by_tma) tma_load_2d(stage + kSaLinOff, &maps.sa, arow, wp.g, &pfull[s]);
         }
         if (!ok) {
           fail();
           // let the tensor copies still in flight land before shared memory is released
-          for (int64_t j = (produced > kStages ? produced - kStages : 0); j < produced; ++j)
-            (void)mbar_wait(&pfull[j % kStages], static_cast<uint32_t>((j / kStages) & 1), nullptr);
+          for (int64_t j = (ls > kNP ? ls - kNP : 0); j < ls; ++j)
+            (void)mbar_wait(&pfull[j % kNP], static_cast<uint32_t>((j / kNP) & 1), nullptr);
         }
       }
     } else if (warp == 1) {
       if (lane == 0 && rank == 0) {
         // ============================================================ MMA issuer (leader)
+        // The peer CTA arrives on mfull (after its proxy fence) and on tempty
+        // (after tcgen05.wait::ld and the tcgen05 fence); both are waited on
+        // with CTA-scope acquire: a cluster-scope acquire costs hundreds of
+        // cycles per wait on B200 and orders nothing more here.
         int64_t last_mma = -1;
         bool ok = true;
-        for (int64_t it = 0; ok && it < iters; ++it) {
-          const int s = static_cast<int>(it % kStages), b = static_cast<int>(it & 1);
-          const uint32_t ph = static_cast<uint32_t>((it / kStages) & 1);
-          if (!mbar_wait(&lfull[s], ph, abort_flag) ||
-              !mbar_wait_cluster(&mfull[s], ph, abort_flag)) {
+        RingPos ur;
+        for (int64_t it = 0; ok && it < iters; ++it, ur.next(kNU)) {
+          const int u = ur.idx, b = static_cast<int>(it & 1);
+          const uint32_t ph = ur.phase;
+          if (!mbar_wait(&ufull[u], ph, abort_flag) ||
+              !mbar_wait(&mfull[u], ph, abort_flag)) {
             ok = false;
             break;
           }
-          const uint32_t a_addr = smem_addr(stages + s * kStageBytes);
+          const uint32_t a_addr = smem_addr(uring + u * kUSlot);
           const uint64_t adesc = smem_desc_k_sw128(a_addr);
 #pragma unroll 1
           for (int h = 0; h < 2; ++h) {
-            if (!mbar_wait_cluster(&tempty[2 * b + h], static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
-                                   abort_flag)) {
+            if (!mbar_wait(&tempty[2 * b + h], static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
+                           abort_flag)) {
               ok = false;
               break;
             }
@@ -538,7 +550,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             tc_commit_pair_multicast(&tfull[2 * b + h], 0x3);
           }
           if (!ok) break;
-          tc_commit_pair_multicast(&empty[s], 0x3);
+          tc_commit_pair_multicast(&uempty[u], 0x3);
           last_mma = it;
         }
         if (!ok) fail();
@@ -554,24 +566,45 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       w.start(p);
       float sa_d = (!p.sa_by_tma && iters > 0) ? sa_direct_load(p, w, rank, lt) : 0.f;
       const uint32_t mfull_leader = cluster_map(&mfull[0], 0);
-      for (int64_t it = 0; it < iters; ++it) {
-        const int s = static_cast<int>(it % kStages);
+      RingPos ur, sr, pr;   // operand, scale and packed rings
+      for (int64_t it = 0; it < iters; ++it, ur.next(kNU), sr.next(kNS)) {
+        const int u = ur.idx, sl = sr.idx;
+        const bool int4_group = w.g < p.G - 1;
+        const RingPos p0 = pr;
+        RingPos p1 = pr;
+        p1.next(kNP);
+        const int s0 = p0.idx, s1 = p1.idx;
         TileWalk wn = w;
         wn.next(p);
-        const bool ok = mbar_wait(&pfull[s], static_cast<uint32_t>((it / kStages) & 1), abort_flag);
-        if (named_bar_any(kBarUnpack, kUnpackThreads, !ok)) {
-          fail();
+        bool ok = mbar_wait(&uempty[u], ur.phase ^ 1u, abort_flag) &&
+                  mbar_wait(&sempty[sl], sr.phase ^ 1u, abort_flag) &&
+                  mbar_wait(&pfull[s0], p0.phase, abort_flag);
+        if (ok && !int4_group) ok = mbar_wait(&pfull[s1], p1.phase, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) fail();
           break;
         }
-        uint8_t *stage = stages + s * kStageBytes;
-        unpack_stage(p, w, lt, stage, sa_d);
+        const uint8_t *pk = pring + s0 * kPSlot;
+        uint8_t *op = uring + u * kUSlot;
+        if (int4_group)
+          unpack_int4(lt, pk, op);
+        else
+          copy_int8(lt, pk, pring + s1 * kPSlot, op);
+        layout_scales(p, lt, pk, sring + sl * kSSlot, sa_d);
         if (!p.sa_by_tma && it + 1 < iters) sa_d = sa_direct_load(p, wn, rank, lt);
         fence_proxy_async_smem();
-        named_bar_sync(kBarUnpack, kUnpackThreads);
-        if (lt == 0) {
-          mbar_arrive(&lfull[s]);
-          if (rank == 1) mbar_arrive_cluster(mfull_leader + 8u * s);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&pempty[s0]);
+          if (!int4_group) mbar_arrive(&pempty[s1]);
+          mbar_arrive(&sfull[sl]);
+          if (rank == 0)
+            mbar_arrive(&ufull[u]);
+          else
+            mbar_arrive_remote(mfull_leader + 8u * u);
         }
+        pr = p1;
+        if (!int4_group) pr.next(kNP);
         w = wn;
       }
     }

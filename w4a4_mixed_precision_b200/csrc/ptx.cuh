@@ -66,10 +66,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Slow path of mbar_wait: keeps polling, and gives up after kWaitLimitNs or
+// once `abort_flag` (shared memory) becomes non-zero. Kept out of line so that
+// the timer read never lands on the fast path.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity,
+                                            const volatile int *abort_flag) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (abort_flag != nullptr && *abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+  }
+}
+
 // Waits for the phase with the given parity to complete. Returns false if the
 // wait ran past kWaitLimitNs or `abort_flag` (shared memory) became non-zero.
+// A phase that has already completed costs about 70 cycles on B200 (a single
+// try_wait is 20; keeping the timed loop inline costs about 160).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           const volatile int *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag);
+}
+
+// The same wait with the slow path inline, for code whose live registers
+// leave no room for a call (about 160 cycles when the phase has completed).
+__device__ __forceinline__ bool mbar_wait_inline(uint64_t *bar, uint32_t parity,
+                                                 const volatile int *abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
@@ -241,6 +266,15 @@ __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_add
                : "memory");
 }
 
+// Arrive on an mbarrier of another CTA of the cluster with the default
+// (release, CTA-scope) semantics. Used after fence.proxy.async by threads that
+// wrote a 2-SM MMA's operands into their own CTA's shared memory: the leader's
+// MMA reads them through the async proxy. A cluster-scope release costs about
+// 1 us more per arrival on B200.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_addr,
                                                               uint32_t bytes) {
   asm volatile(
@@ -262,10 +296,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
   return ok != 0;
 }
 
-// Bounded wait for a barrier that other CTAs of the cluster arrive on.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
-                                                  const volatile int *abort_flag) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait_cluster_slow(uint64_t *bar, uint32_t parity,
+                                                    const volatile int *abort_flag) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
@@ -274,6 +306,14 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
       if (global_timer_ns() - t0 > kWaitLimitNs) return false;
     }
   }
+}
+
+// Bounded wait with cluster-scope acquire, for a barrier whose arrivals
+// release writes that this thread's own generic loads must see.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
+                                                  const volatile int *abort_flag) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  return mbar_wait_cluster_slow(bar, parity, abort_flag);
 }
 
 __device__ __forceinline__ void cluster_sync() {
@@ -428,6 +468,17 @@ __device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
 __device__ __forceinline__ uint32_t pack_half2_rn(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Exact int32 -> fp32 conversion for |p| < 2^22, as bits: keeps the low 23
+// bits of p with bit 22 flipped (that is p + 2^22 mod 2^23) under the exponent
+// of 2^23, so the float equals 1.5*2^23 + p. One LOP3 (select by the mask
+// 0x007FFFFF between p ^ 0x4B400000 and 0x4B400000), which runs on the
+// integer ALU pipe and leaves the FMA pipe to the scale arithmetic.
+__device__ __forceinline__ uint32_t biased_float_bits(uint32_t p) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(r) : "r"(p), "r"(0x007FFFFFu), "r"(0x4B400000u));
   return r;
 }
 
