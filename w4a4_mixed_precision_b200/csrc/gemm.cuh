@@ -15,12 +15,10 @@
 // Structure. A cluster of two CTAs on two SMs owns a 256x256 output tile: CTA
 // r holds A rows [128r, 128r+128) and W rows [128r, 128r+128) of the tile in
 // its shared memory, and its TMEM receives output rows [128r, 128r+128). Each
-// 128-wide K group is issued as two column halves of 2-SM MMAs (cta_group::2,
-// M=256, N=128, K=32); half h takes W rows [64h, 64h+64) from each CTA, so
-// accumulator column j of half h is tile column 64h + (j mod 64) + 128*(j/64).
-// Two groups in flight x two halves gives four 128-column accumulators per
-// CTA, and the drain hands each half back as soon as it has read it. The pairs
-// are persistent over tiles (m fastest).
+// 128-wide K group is four 2-SM MMAs (cta_group::2, M=256, N=256, K=32): the
+// B operand is CTA 0's 128 W rows followed by CTA 1's, so accumulator column j
+// is tile column j. Two groups are in flight in two 256-column TMEM
+// accumulators per CTA. The pairs are persistent over tiles (m fastest).
 //
 // Three shared-memory rings decouple the stages, so that no stage holds a
 // buffer longer than its own step needs:
@@ -35,23 +33,22 @@
 // Roles in each CTA:
 //
 //   producer (warp 0, lane 0)  TMA copies into the packed ring.
-//   warp 1, lane 0     (leader CTA) per group and half: 4 x 2-SM MMA into a
-//                      128-column TMEM accumulator, commit to both CTAs' "half
-//                      full" barrier; after both halves commit to both CTAs'
-//                      "operands free" barrier.
+//   warp 1, lane 0     (leader CTA) per group: 4 x 2-SM MMA into a 256-column
+//                      TMEM accumulator, then commits to both CTAs'
+//                      "accumulator full" and "operands free" barriers.
 //   unpack warps 2..7  expand each nibble of the packed tiles to a byte
 //                      holding 16*q (x << 4 & 0xF0 / x & 0xF0), store K-major
 //                      with the 128-byte swizzle (the INT8 group is copied),
 //                      and lay the scales out for the drain; then one thread
 //                      signals "operands ready" locally and, from the peer CTA,
 //                      to the leader.
-//   drain warps 8..15  warps 8..11 drain accumulator half 0 and 12..15 half 1:
-//                      each thread reads one TMEM lane (one output row) with
-//                      the 32x32b shape, 16 columns per load, accumulates
-//                      sa*sw*P into 128 fp32 registers, and each half is
-//                      handed back to the MMA as soon as its four warps have
-//                      read it (one arrival per CTA, on the leader). After the
-//                      last group of a tile: fp16 stores.
+//   drain warps 8..15  warps 8..11 drain accumulator columns [0, 128) and
+//                      12..15 columns [128, 256): each thread reads one TMEM
+//                      lane (one output row) with the 32x32b shape, 16 columns
+//                      per load, accumulates sa*sw*P into 128 fp32 registers,
+//                      and arrives on the leader's "accumulator free" barrier
+//                      once its loads are done. After the last group of a
+//                      tile: fp16 stores.
 //
 // Exact integer -> float: F = float with the low 23 bits of P + 2^22 under the
 // exponent of 2^23 equals 1.5*2^23 + P exactly for |P| < 2^22 (one LOP3 per
@@ -105,8 +102,8 @@ constexpr uint32_t kSmemBytes = kSOff + kNS * kSSlot + 1024;  // + alignment sla
 constexpr int kPackedChunks = (BM + BW) * 4;                    // 16-B chunks per INT4 group
 constexpr int kChunksPerThread = (kPackedChunks + kUnpackThreads - 1) / kUnpackThreads;
 constexpr int kInt8Chunks = (kABytes + kBBytes) / 16;           // 16-B chunks of an INT8 group
-constexpr int kHalfN = BN / 2;   // columns per MMA / accumulator half
-constexpr uint32_t kIdesc = idesc_i8(kPairM, kHalfN);
+constexpr int kHalfN = BN / 2;   // accumulator columns per drain warp
+constexpr uint32_t kIdesc = idesc_i8(kPairM, BN);
 constexpr float kBiasF = 12582912.0f;
 constexpr int kUnpackRegs = 72;
 constexpr int kDrainRegs = 184;
@@ -199,17 +196,9 @@ __device__ __forceinline__ int64_t pair_iterations(const GemmParams &p) {
 
 // ------------------------------------------------------------------ unpack role
 
-// Tile column of accumulator column c (0..255): c = 128h + j holds the MMA half
-// h column j, which is W row 64h + (j mod 64) of CTA j/64.
-__device__ __forceinline__ int tile_col(int c) {
-  const int h = c >> 7, j = c & 127;
-  return ((j >> 6) << 7) + (h << 6) + (j & 63);
-}
-
-// Scale slot layout: sa by local row (128 floats), then sw by accumulator
-// column (256 floats: entry c holds sw of tile column tile_col(c)), so a drain
-// thread, which owns one row, reads its sa once and the sw of 16 consecutive
-// accumulator columns as four 16-byte broadcast loads.
+// Scale slot layout: sa by local row (128 floats), then sw by tile column (256
+// floats), so a drain thread, which owns one row, reads its sa once and the sw
+// of 16 consecutive columns as four 16-byte broadcast loads.
 // One INT4 group: expands this thread's share of the packed tiles in `pk`
 // into the swizzled int8 operands in `op`.
 __device__ __forceinline__ void unpack_int4(int lt, const uint8_t *pk, uint8_t *op) {
@@ -265,7 +254,7 @@ __device__ __forceinline__ void layout_scales(const GemmParams &p, int lt, const
       const int j = lt - BM + kSwThreads * k;
       if (j < BN)
         reinterpret_cast<float *>(ss + kSwOff)[j] =
-            reinterpret_cast<const float *>(pk + kSwLinOff)[tile_col(j)];
+            reinterpret_cast<const float *>(pk + kSwLinOff)[j];
     }
   }
 }
@@ -306,9 +295,9 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   uint64_t *uempty = mfull + kNU;      // [kNU] MMA commit -> unpackers (both CTAs)
   uint64_t *sfull = uempty + kNU;      // [kNS] scales ready -> drain
   uint64_t *sempty = sfull + kNS;      // [kNS] drain -> unpackers
-  uint64_t *tfull = sempty + kNS;      // [4]   accumulator (buffer b, half h) at 2b+h
-  uint64_t *tempty = tfull + 4;        // [4]   leader only: both CTAs drained (b, h)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 4);
+  uint64_t *tfull = sempty + kNS;      // [2]   accumulator buffer b complete
+  uint64_t *tempty = tfull + 2;        // [2]   leader only: buffer b drained by both CTAs
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   uint8_t *uring = smem + kUOff;
   uint8_t *pring = smem + kPOff;
@@ -331,9 +320,9 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       mbar_init(&sfull[s], kUnpackWarps);    // lane 0 of each unpack warp
       mbar_init(&sempty[s], 8);      // one lane of each drain warp
     }
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 8);      // lane 0 of the half's 4 drain warps in each CTA
+      mbar_init(&tempty[i], 16);     // lane 0 of each of the 8 drain warps in each CTA
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -376,7 +365,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     for (int64_t it = 0; it < iters; ++it, w.next(p), sr.next(kNS)) {
       const int b = static_cast<int>(it & 1), sl = sr.idx;
       const bool ok =
-          mbar_wait_inline(&tfull[2 * b + hh], static_cast<uint32_t>((it >> 1) & 1), abort_flag) &&
+          mbar_wait_inline(&tfull[b], static_cast<uint32_t>((it >> 1) & 1), abort_flag) &&
           mbar_wait_inline(&sfull[sl], sr.phase, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) fail();
@@ -407,7 +396,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
           // 16 consecutive tile columns; N % 8 == 0, so each 4-column store is
           // wholly inside or wholly outside the matrix.
           const int row = w.m0 + BM * rank + lrow;
-          const int col0 = w.n0 + tile_col(hh * kHalfN + 16 * c);
+          const int col0 = w.n0 + hh * kHalfN + 16 * c;
           const int sh = w.g < p.G - 1 ? 8 : 0;
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -440,28 +429,25 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       __syncwarp();
       if (lane == 0) {
         if (rank == 0)
-          mbar_arrive(&tempty[2 * b + hh]);
+          mbar_arrive(&tempty[b]);
         else
-          mbar_arrive_cluster_relaxed(tempty_leader + 8u * (2 * b + hh));
+          mbar_arrive_cluster_relaxed(tempty_leader + 8u * b);
         mbar_arrive(&sempty[sl]);
       }
 
       if (w.g == p.G - 1) {
-        // epilogue: accumulator column 128hh + j is tile column
-        // 64hh + (j mod 64) + 128*(j/64): two runs of 64 columns per row.
+        // epilogue: this thread's 128 columns of its row, 8 per 16-byte store
         const int row = w.m0 + BM * rank + lrow;
         const bool have_y = p.y != nullptr;
 #pragma unroll
-        for (int seg = 0; seg < 2; ++seg)
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const int col = w.n0 + 128 * seg + 64 * hh + 8 * v;
-            const float2 *a = acc + 32 * seg + 4 * v;
-            const bool oky = have_y && row < p.M && col < p.N;
-            st_global_v4_if(p.y + static_cast<int64_t>(oky ? row : 0) * p.N + (oky ? col : 0),
-                            pack_half2_rn(a[0].x, a[0].y), pack_half2_rn(a[1].x, a[1].y),
-                            pack_half2_rn(a[2].x, a[2].y), pack_half2_rn(a[3].x, a[3].y), oky);
-          }
+        for (int v = 0; v < 16; ++v) {
+          const int col = w.n0 + kHalfN * hh + 8 * v;
+          const float2 *a = acc + 4 * v;
+          const bool oky = have_y && row < p.M && col < p.N;
+          st_global_v4_if(p.y + static_cast<int64_t>(oky ? row : 0) * p.N + (oky ? col : 0),
+                          pack_half2_rn(a[0].x, a[0].y), pack_half2_rn(a[1].x, a[1].y),
+                          pack_half2_rn(a[2].x, a[2].y), pack_half2_rn(a[3].x, a[3].y), oky);
+        }
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
       }
@@ -531,32 +517,26 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             ok = false;
             break;
           }
+          if (!mbar_wait(&tempty[b], static_cast<uint32_t>(((it >> 1) & 1) ^ 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
           const uint32_t a_addr = smem_addr(uring + u * kUSlot);
           const uint64_t adesc = smem_desc_k_sw128(a_addr);
-#pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
-            if (!mbar_wait(&tempty[2 * b + h], static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
-                           abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after_sync();
-            // half h: W rows [64h, 64h+64) of each CTA's tile
-            const uint64_t bdesc = smem_desc_k_sw128(a_addr + kABytes + h * 64 * 128);
-            const uint32_t d = tbase + b * BN + h * kHalfN;
+          const uint64_t bdesc = smem_desc_k_sw128(a_addr + kABytes);
+          const uint32_t d = tbase + b * BN;
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
-            tc_commit_pair_multicast(&tfull[2 * b + h], 0x3);
-          }
-          if (!ok) break;
+          for (int k = 0; k < 4; ++k)
+            mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
+          tc_commit_pair_multicast(&tfull[b], 0x3);
           tc_commit_pair_multicast(&uempty[u], 0x3);
           last_mma = it;
         }
         if (!ok) fail();
         // nothing may still write TMEM when it is released
         if (last_mma >= 0)
-          (void)mbar_wait(&tfull[2 * (last_mma & 1) + 1],
+          (void)mbar_wait(&tfull[last_mma & 1],
                           static_cast<uint32_t>((last_mma >> 1) & 1), nullptr);
       }
     } else {
