@@ -50,10 +50,12 @@
 //                      once its loads are done. After the last group of a
 //                      tile: fp16 stores.
 //
-// Exact integer -> float: F = float with the low 23 bits of P + 2^22 under the
-// exponent of 2^23 equals 1.5*2^23 + P exactly for |P| < 2^22 (one LOP3 per
-// element on the integer pipe; the alternative of pre-filling TMEM with that
-// bias doubles the TMEM traffic).
+// Exact integer -> float without a conversion instruction: every accumulator
+// starts at the int32 0x4B400000 (the bits of C = 1.5*2^23) and the MMAs add
+// the group's partial P onto it, so the int32 in TMEM is the bit pattern of
+// the float C + P, exact for |P| < 2^22 (INT4 groups: |256 P| <= 1.6e6; INT8
+// group: |P| <= 2.1e6). The drain re-arms each 16-column chunk with a TMEM
+// store as soon as it has loaded it.
 // Dequantisation: with sa' = sa truncated to 22 significant bits, C*sa' is
 // exact for C = 1.5*2^23, so t = fma(F, sa', -C*sa') = round(P*sa') in one
 // instruction, then acc = fma(t, sw, acc); both run as packed f32x2 pairs.
@@ -104,6 +106,7 @@ constexpr int kChunksPerThread = (kPackedChunks + kUnpackThreads - 1) / kUnpackT
 constexpr int kInt8Chunks = (kABytes + kBBytes) / 16;           // 16-B chunks of an INT8 group
 constexpr int kHalfN = BN / 2;   // accumulator columns per drain warp
 constexpr uint32_t kIdesc = idesc_i8(kPairM, BN);
+constexpr uint32_t kBias = 0x4B400000u;  // bits of 1.5 * 2^23
 constexpr float kBiasF = 12582912.0f;
 constexpr int kUnpackRegs = 72;
 constexpr int kDrainRegs = 184;
@@ -337,6 +340,20 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   const uint32_t tbase = *tmem_slot;
   const int64_t iters = pair_iterations(p);
 
+  // Both accumulators start at the conversion bias (see the drain), and every
+  // MMA accumulates onto what TMEM holds.
+  if (warp >= 8) {
+    const uint32_t lanes = tbase + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
+                           ((warp - 8) >> 2) * kHalfN;
+#pragma unroll
+    for (int c = 0; c < 16; ++c)   // buffer c/8, 16-column chunk c%8 of this warp's half
+      tmem_st_x16_fill(lanes + (c >> 3) * BN + 16 * (c & 7), kBias);
+    tmem_st_wait();
+  }
+  tc_fence_before_sync();
+  cluster_sync();
+  tc_fence_after_sync();
+
   auto fail = [&](void) {
     report_status(6 /* ATOM_ERR_TIMEOUT */);
     *abort_flag = 1;
@@ -391,6 +408,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       for (int c = 0; c < 8; ++c) {   // 16 accumulator columns per chunk
         uint32_t(&r)[16] = (c & 1) ? rb : ra;
         uint32_t(&rn)[16] = (c & 1) ? ra : rb;
+        tmem_st_x16_fill(tcol + 16 * c, kBias);   // re-arm these columns for the next use
         if (c + 1 < 8) tmem_ld_x16(tcol + 16 * (c + 1), rn);
         if (kPartials) {
           // 16 consecutive tile columns; N % 8 == 0, so each 4-column store is
@@ -404,27 +422,27 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             const bool okp = row < p.M && col < p.N;
             int32_t *dst = p.partials +
                            (static_cast<int64_t>(w.g) * p.M + (okp ? row : 0)) * p.N + (okp ? col : 0);
-            st_global_v4_if(dst, static_cast<uint32_t>(static_cast<int32_t>(r[4 * v]) >> sh),
-                            static_cast<uint32_t>(static_cast<int32_t>(r[4 * v + 1]) >> sh),
-                            static_cast<uint32_t>(static_cast<int32_t>(r[4 * v + 2]) >> sh),
-                            static_cast<uint32_t>(static_cast<int32_t>(r[4 * v + 3]) >> sh), okp);
+            st_global_v4_if(dst, static_cast<uint32_t>(static_cast<int32_t>(r[4 * v] - kBias) >> sh),
+                            static_cast<uint32_t>(static_cast<int32_t>(r[4 * v + 1] - kBias) >> sh),
+                            static_cast<uint32_t>(static_cast<int32_t>(r[4 * v + 2] - kBias) >> sh),
+                            static_cast<uint32_t>(static_cast<int32_t>(r[4 * v + 3] - kBias) >> sh),
+                            okp);
           }
         }
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const float4 s4 = sw4[4 * c + v];
           float2 *a = acc + 8 * c + 2 * v;
-          const float2 f0 = make_float2(__uint_as_float(biased_float_bits(r[4 * v])),
-                                        __uint_as_float(biased_float_bits(r[4 * v + 1])));
-          const float2 f1 = make_float2(__uint_as_float(biased_float_bits(r[4 * v + 2])),
-                                        __uint_as_float(biased_float_bits(r[4 * v + 3])));
+          const float2 f0 = make_float2(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]));
+          const float2 f1 = make_float2(__uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
           a[0] = f2_fma(f2_fma(f0, sa2, nc2), make_float2(s4.x, s4.y), a[0]);
           a[1] = f2_fma(f2_fma(f1, sa2, nc2), make_float2(s4.z, s4.w), a[1]);
         }
         if (c + 1 < 8) tmem_ld_wait(rn);
       }
-      // this warp's lanes of the half are in registers: hand them back, and
-      // the group's scales with them
+      // this warp's lanes of the half are in registers and re-armed: hand them
+      // back, and the group's scales with them
+      tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) {
@@ -528,7 +546,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
           const uint32_t d = tbase + b * BN;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, k > 0 ? 1u : 0u);
+            mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, 1u);
           tc_commit_pair_multicast(&tfull[b], 0x3);
           tc_commit_pair_multicast(&uempty[u], 0x3);
           last_mma = it;

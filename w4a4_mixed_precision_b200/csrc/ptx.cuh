@@ -396,19 +396,12 @@ __device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_st_16x256b_x4_fill(uint32_t taddr, uint32_t v) {
+// Writes `v` to 16 consecutive columns of this thread's TMEM lane (the store
+// counterpart of tmem_ld_x16).
+__device__ __forceinline__ void tmem_st_x16_fill(uint32_t taddr, uint32_t v) {
   asm volatile(
-      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], "
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
-      "r"(v)
-      : "memory");
-}
-
-// Writes the same register to every element a 16x256b.x2 load would read.
-__device__ __forceinline__ void tmem_st_16x256b_x2_fill(uint32_t taddr, uint32_t v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.16x256b.x2.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(
-          taddr),
       "r"(v)
       : "memory");
 }
