@@ -346,8 +346,8 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     const uint32_t lanes = tbase + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
                            ((warp - 8) >> 2) * kHalfN;
 #pragma unroll
-    for (int c = 0; c < 16; ++c)   // buffer c/8, 16-column chunk c%8 of this warp's half
-      tmem_st_x16_fill(lanes + (c >> 3) * BN + 16 * (c & 7), kBias);
+    for (int c = 0; c < 64; ++c)   // buffer c/32, 4-column chunk c%32 of this warp's half
+      tmem_st_x4_fill(lanes + (c >> 5) * BN + 4 * (c & 31), kBias);
     tmem_st_wait();
   }
   tc_fence_before_sync();
@@ -408,7 +408,9 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       for (int c = 0; c < 8; ++c) {   // 16 accumulator columns per chunk
         uint32_t(&r)[16] = (c & 1) ? rb : ra;
         uint32_t(&rn)[16] = (c & 1) ? ra : rb;
-        tmem_st_x16_fill(tcol + 16 * c, kBias);   // re-arm these columns for the next use
+#pragma unroll
+        for (int e = 0; e < 4; ++e)   // re-arm these columns for the next use
+          tmem_st_x4_fill(tcol + 16 * c + 4 * e, kBias);
         if (c + 1 < 8) tmem_ld_x16(tcol + 16 * (c + 1), rn);
         if (kPartials) {
           // 16 consecutive tile columns; N % 8 == 0, so each 4-column store is

@@ -396,14 +396,12 @@ __device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
-// Writes `v` to 16 consecutive columns of this thread's TMEM lane (the store
-// counterpart of tmem_ld_x16).
-__device__ __forceinline__ void tmem_st_x16_fill(uint32_t taddr, uint32_t v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
-      "r"(v)
-      : "memory");
+// Writes `v` to 4 consecutive columns of this thread's TMEM lane. (The wider
+// forms take one register per column, which the compiler materialises as
+// copies of `v`: 16 of them overflow the drain's register budget.)
+__device__ __forceinline__ void tmem_st_x4_fill(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %1, %1, %1};" ::"r"(taddr), "r"(v)
+               : "memory");
 }
 
 __device__ __forceinline__ void tmem_st_wait() {
