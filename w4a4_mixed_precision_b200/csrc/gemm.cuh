@@ -54,8 +54,8 @@
 // starts at the int32 0x4B400000 (the bits of C = 1.5*2^23) and the MMAs add
 // the group's partial P onto it, so the int32 in TMEM is the bit pattern of
 // the float C + P, exact for |P| < 2^22 (INT4 groups: |256 P| <= 1.6e6; INT8
-// group: |P| <= 2.1e6). The drain re-arms each 16-column chunk with a TMEM
-// store as soon as it has loaded it.
+// group: |P| <= 2.1e6). The drain re-arms its columns with TMEM stores once
+// it has loaded them.
 // Dequantisation: with sa' = sa truncated to 22 significant bits, C*sa' is
 // exact for C = 1.5*2^23, so t = fma(F, sa', -C*sa') = round(P*sa') in one
 // instruction, then acc = fma(t, sw, acc); both run as packed f32x2 pairs.
@@ -408,9 +408,6 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       for (int c = 0; c < 8; ++c) {   // 16 accumulator columns per chunk
         uint32_t(&r)[16] = (c & 1) ? rb : ra;
         uint32_t(&rn)[16] = (c & 1) ? ra : rb;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)   // re-arm these columns for the next use
-          tmem_st_x4_fill(tcol + 16 * c + 4 * e, kBias);
         if (c + 1 < 8) tmem_ld_x16(tcol + 16 * (c + 1), rn);
         if (kPartials) {
           // 16 consecutive tile columns; N % 8 == 0, so each 4-column store is
@@ -442,8 +439,11 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         }
         if (c + 1 < 8) tmem_ld_wait(rn);
       }
-      // this warp's lanes of the half are in registers and re-armed: hand them
-      // back, and the group's scales with them
+      // this warp's lanes of the half are in registers: re-arm them with the
+      // bias (in one burst, off the arithmetic's path) and hand them back, and
+      // the group's scales with them
+#pragma unroll
+      for (int e = 0; e < kHalfN / 4; ++e) tmem_st_x4_fill(tcol + 4 * e, kBias);
       tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
