@@ -60,18 +60,24 @@ def _kernel_source_hash() -> str:
 
 
 def _profiled_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch (read + write) from the committed ncu summary
+    profiles/traffic.md, if it was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
     try:
         with open(path) as f:
-            d = json.load(f)
-    except (OSError, ValueError):
+            lines = f.read().splitlines()
+    except OSError:
         return None
-    e = d.get(kernel)
-    if not e or e.get("source_hash") != _kernel_source_hash():
-        return None
-    return e.get("dram_bytes_per_launch")
+    for line in lines:
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 5 and cells[0] == kernel:
+            if cells[1] != _kernel_source_hash():
+                return None
+            try:
+                return int(cells[4])
+            except ValueError:
+                return None
+    return None
 
 
 # ----------------------------------------------------------------------------- clocks
