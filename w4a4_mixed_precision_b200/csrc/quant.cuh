@@ -190,11 +190,14 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
   }
 
   int64_t done = 0;  // rows this CTA has finished
+  // Stage slot and barrier parity of row i and of row i-1, advanced by
+  // counting (no division on the per-row path).
+  int s = 0, s_prev = 0;
+  uint32_t ph = 0, ph_prev = 0;
   for (int64_t i = 0;; ++i) {
     const int64_t r = blockIdx.x + i * grid;
     if (r >= rows) break;
-    const int s = static_cast<int>(i % stages_n);
-    if (!mbar_wait(&full[s], static_cast<uint32_t>((i / stages_n) & 1), &flags[1])) {
+    if (!mbar_wait(&full[s], ph, &flags[1])) {
       if (lane == 0) {
         report_status(6 /* ATOM_ERR_TIMEOUT */);
         flags[1] = 1;
@@ -202,6 +205,9 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
       break;
     }
     const uint8_t *row = stage_base + s * L.row_bytes;
+    uint8_t *q4_r = q4 + r * q4_row;
+    int8_t *q8_r = q8 + r * 128;
+    float *scales_r = scales + r;
 
     for (int gb = 0; gb < G; gb += 32) {
       const int g = gb + warp * 4 + team;
@@ -245,7 +251,7 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
         const uint32_t od1 = low_bytes4(b[9], b[11], b[13], b[15]);
         const uint32_t lo = (ev0 & 0x0F0F0F0Fu) | ((od0 << 4) & 0xF0F0F0F0u);
         const uint32_t hi = (ev1 & 0x0F0F0F0Fu) | ((od1 << 4) & 0xF0F0F0F0u);
-        *reinterpret_cast<uint2 *>(q4 + r * q4_row + g * 64 + sub * 8) =
+        *reinterpret_cast<uint2 *>(q4_r + g * 64 + sub * 8) =
             make_uint2(__byte_perm(lo, hi, sel_lo), __byte_perm(lo, hi, sel_hi));
       } else {
         uint4 o;
@@ -253,9 +259,9 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
         o.y = low_bytes4(b[4], b[5], b[6], b[7]);
         o.z = low_bytes4(b[8], b[9], b[10], b[11]);
         o.w = low_bytes4(b[12], b[13], b[14], b[15]);
-        *reinterpret_cast<uint4 *>(q8 + r * 128 + sub * 16) = o;
+        *reinterpret_cast<uint4 *>(q8_r + sub * 16) = o;
       }
-      if (sub == 0) scales[static_cast<int64_t>(g) * rows + r] = scale;
+      if (sub == 0) scales_r[static_cast<int64_t>(g) * rows] = scale;
     }
 
     __syncwarp();
@@ -265,18 +271,22 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     // Refill the stage of the previous row: one row of slack, so the issuing
     // thread rarely waits for the slowest warp.
     if (tid == 0 && i >= 1) {
-      const int64_t j = i - 1;
-      const int64_t nr = blockIdx.x + (j + stages_n) * grid;
+      const int64_t nr = blockIdx.x + (i - 1 + stages_n) * grid;
       if (nr < rows) {
-        const int sj = static_cast<int>(j % stages_n);
-        if (!mbar_wait(&empty[sj], static_cast<uint32_t>((j / stages_n) & 1), &flags[1])) {
+        if (!mbar_wait(&empty[s_prev], ph_prev, &flags[1])) {
           report_status(6 /* ATOM_ERR_TIMEOUT */);
           flags[1] = 1;
           break;
         }
-        mbar_arrive_expect_tx(&full[sj], L.row_bytes);
-        bulk_load(stage_base + sj * L.row_bytes, x + nr * ld, L.row_bytes, &full[sj]);
+        mbar_arrive_expect_tx(&full[s_prev], L.row_bytes);
+        bulk_load(stage_base + s_prev * L.row_bytes, x + nr * ld, L.row_bytes, &full[s_prev]);
       }
+    }
+    s_prev = s;
+    ph_prev = ph;
+    if (++s == stages_n) {
+      s = 0;
+      ph ^= 1u;
     }
   }
 
