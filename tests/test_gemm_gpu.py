@@ -62,7 +62,9 @@ def test_partials_bit_exact_and_output_within_tolerance(c_oracle, name):
     assert mism.size == 0, f"{len(mism)} partial mismatches, first {mism[:3].tolist()}"
     assert y_rel_err(y, Y64) <= Y_TOL
     assert y_rel_err(y2, Y64) <= Y_TOL
-    assert np.array_equal(y.view(np.uint16), y2.view(np.uint16))   # same mainloop, same Y
+    if atom.atom_gemm_workspace_bytes(A.shape[0], W.shape[0], A.shape[1]) == 0:
+        # no K split: the same mainloop in the same order gives the same Y
+        assert np.array_equal(y.view(np.uint16), y2.view(np.uint16))
 
 
 def test_lossless_integers_give_the_exact_integer_matmul(c_oracle):
@@ -155,3 +157,43 @@ def test_back_to_back_calls_are_deterministic():
     y2 = atom.atom_w4a4_gemm(qa, qw, K)
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("M,N,K,seed", [(64, 4096, 4096, 21), (40, 520, 2048, 22),
+                                        (1, 256, 32768, 23), (130, 1024, 1152, 24)])
+def test_split_k_output_matches_oracle_and_unsplit(c_oracle, M, N, K, seed):
+    """Small-M shapes split K across CTA pairs (fp32 partial tiles in the
+    workspace, summed in split order). Y must be within tolerance of the
+    oracle on every row, with and without the split."""
+    ws = atom.atom_gemm_workspace_bytes(M, N, K)
+    assert ws > 0 and ws % (4 * M * N) == 0        # these shapes do split
+    A, W, idx = inputs.random_case(seed, M, N, K, dist="t", param=4.0, outlier_factor=30.0)
+    qa, qw = quant_dev(A, idx), quant_dev(W, idx, weights=True)
+    y_split = atom.atom_w4a4_gemm(qa, qw, K).cpu().numpy()
+    y_plain = atom.atom_w4a4_gemm(qa, qw, K, split=False).cpu().numpy()
+    ra, rw = c_oracle.quantize(A, idx), c_oracle.quantize(W, idx)
+    Y64 = c_oracle.gemm(*ra, *rw, K)
+    for y in (y_split, y_plain):
+        err = y_rel_err(y, Y64)
+        assert err <= Y_TOL, err
+
+
+def test_split_k_is_deterministic_and_ignores_a_short_workspace():
+    M, N, K = 64, 4096, 4096
+    A, W, idx = inputs.random_case(25, M, N, K)
+    qa, qw = quant_dev(A, idx), quant_dev(W, idx, weights=True)
+    y1 = atom.atom_w4a4_gemm(qa, qw, K).clone()
+    y2 = atom.atom_w4a4_gemm(qa, qw, K)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    # a workspace one byte short of the size asked for runs without the split
+    short = torch.empty(atom.atom_gemm_workspace_bytes(M, N, K) - 1, dtype=torch.uint8,
+                        device="cuda")
+    y3 = atom.atom_w4a4_gemm(qa, qw, K, workspace=short)
+    y4 = atom.atom_w4a4_gemm(qa, qw, K, split=False)
+    torch.cuda.synchronize()
+    assert torch.equal(y3.view(torch.int16), y4.view(torch.int16))
+
+
+def test_large_shapes_do_not_split():
+    assert atom.atom_gemm_workspace_bytes(8192, 28672, 8192) == 0
+    assert atom.atom_gemm_workspace_bytes(4096, 11008, 4096) == 0

@@ -147,17 +147,33 @@ def atom_quant_weights(w: torch.Tensor, outlier_idx: torch.Tensor,
     return _quant("atom_quant_weights", w, outlier_idx, out, stream)
 
 
+def gemm_workspace(M: int, N: int, K: int, device) -> Optional[torch.Tensor]:
+    """Scratch for atom_w4a4_gemm on this shape (None when it needs none)."""
+    n = atom_gemm_workspace_bytes(M, N, K)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n > 0 else None
+
+
 def atom_w4a4_gemm(qa: Quantized, qw: Quantized, K: int, y: Optional[torch.Tensor] = None,
-                   stream=None) -> torch.Tensor:
-    """Y fp16 [M, N] = sum_g sa*sw*P_g (see include/atom.h)."""
+                   stream=None, workspace: Optional[torch.Tensor] = None,
+                   split: bool = True) -> torch.Tensor:
+    """Y fp16 [M, N] = sum_g sa*sw*P_g (see include/atom.h).
+
+    `workspace` (uint8 CUDA tensor) is the scratch a split-K launch uses; when it
+    is None and `split` is true, one of atom_gemm_workspace_bytes() bytes is
+    allocated here. `split=False` runs without a workspace (no K split)."""
     M, N = qa.rows, qw.rows
+    dev = qa.q4.device
     if y is None:
-        y = torch.empty((M, N), dtype=torch.float16, device=qa.q4.device)
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    if workspace is None and split:
+        workspace = gemm_workspace(M, N, K, dev)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None or not split else (
+        _dev(workspace, torch.uint8, "workspace"), workspace.numel())
     st = lib().atom_w4a4_gemm(
         _dev(qa.q4, torch.uint8, "qa4"), _dev(qa.q8, torch.int8, "qa8"),
         _dev(qa.scales, torch.float32, "sa"), _dev(qw.q4, torch.uint8, "qw4"),
         _dev(qw.q8, torch.int8, "qw8"), _dev(qw.scales, torch.float32, "sw"),
-        _dev(y, torch.float16, "y"), M, N, K, N_OUTLIER, GROUP, None, 0, _stream(stream))
+        _dev(y, torch.float16, "y"), M, N, K, N_OUTLIER, GROUP, ws_ptr, ws_bytes, _stream(stream))
     _check("atom_w4a4_gemm", st)
     return y
 

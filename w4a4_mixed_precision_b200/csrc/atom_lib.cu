@@ -151,10 +151,30 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// K splits for a GEMM whose output tiles would leave most CTA pairs idle
+// (small M: decode): as many as fill the pairs, at least kMinGroupsPerSplit
+// groups of 128 each. 1 = no split.
+constexpr int kMinGroupsPerSplit = 4;
+constexpr int kMaxSplits = 16;
+
+int gemm_splits(int64_t M, int64_t N, int64_t K, int pairs) {
+  using namespace atomk::gemm_cfg;
+  const int64_t tiles = ((M + kPairM - 1) / kPairM) * ((N + BN - 1) / BN);
+  if (tiles <= 0 || 2 * tiles >= pairs) return 1;
+  int64_t s = pairs / tiles;
+  const int64_t by_k = (K / 128) / kMinGroupsPerSplit;
+  if (s > by_k) s = by_k;
+  if (s > kMaxSplits) s = kMaxSplits;
+  return s < 2 ? 1 : static_cast<int>(s);
+}
+
+atom_status_t gemm_pairs(DeviceState *dev, bool pmode, int *pairs);
+
 atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa,
                           const uint8_t *qw4, const int8_t *qw8, const float *sw, void *y,
                           int32_t *partials, int64_t M, int64_t N, int64_t K, int32_t n_outlier,
-                          int32_t group, atom_stream_t stream) {
+                          int32_t group, void *workspace, size_t workspace_bytes,
+                          atom_stream_t stream) {
   if (M < 0 || N < 0) return ATOM_ERR_INVALID_ARG;
   atom_status_t st = check_method_params(K, n_outlier, group);
   if (st != ATOM_OK) return st;
@@ -175,30 +195,8 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
 
   using namespace atomk::gemm_cfg;
   const bool pmode = partials != nullptr;
-  if (!dev->gemm_attr[pmode]) {
-    std::lock_guard<std::mutex> lock(g_mutex);
-    const void *fn = pmode ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<true>)
-                           : reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<false>);
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess)
-      return ATOM_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * dev->sm_count, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 2;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg) != cudaSuccess || clusters < 1)
-      clusters = dev->sm_count / 2;
-    dev->gemm_clusters[pmode] = clusters;
-    dev->gemm_attr[pmode] = true;
-  }
+  int pairs = 0;
+  if ((st = gemm_pairs(dev, pmode, &pairs)) != ATOM_OK) return st;
 
   const int64_t G = K / 128;
   atomk::GemmMaps maps;
@@ -233,16 +231,66 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   p.m_tiles = static_cast<int>((M + kPairM - 1) / kPairM);
   p.n_tiles = static_cast<int>((N + BN - 1) / BN);
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
-  if (tiles > INT32_MAX) return ATOM_ERR_SHAPE;
+  // Split K only for the output, with a workspace large enough for the partials.
+  int splits = pmode ? 1 : gemm_splits(M, N, K, pairs);
+  if (splits > 1 && (workspace == nullptr ||
+                     workspace_bytes < static_cast<size_t>(splits) * M * N * sizeof(float) ||
+                     !aligned(workspace, 16)))
+    splits = 1;
+  if (tiles * splits > INT32_MAX) return ATOM_ERR_SHAPE;
   p.tiles = static_cast<int>(tiles);
-  const int64_t pairs = tiles < dev->gemm_clusters[pmode] ? tiles : dev->gemm_clusters[pmode];
-  const int grid = static_cast<int>(2 * pairs);   // CTA pairs (cluster of 2)
+  p.splits = splits;
+  p.items = static_cast<int>(tiles * splits);
+  p.ws = splits > 1 ? static_cast<float *>(workspace) : nullptr;
+  const int64_t used = p.items < pairs ? p.items : pairs;
+  const int grid = static_cast<int>(2 * used);   // CTA pairs (cluster of 2)
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (pmode)
     atomk::w4a4_gemm_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
   else
     atomk::w4a4_gemm_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
-  return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return ATOM_ERR_CUDA;
+  if (splits > 1) {
+    const int64_t count8 = M * N / 8;
+    int64_t blocks = (count8 + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(dev->sm_count) * 8;
+    if (blocks > cap) blocks = cap;
+    atomk::splitk_reduce_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
+        p.ws, static_cast<__half *>(y), count8, M * N, splits);
+    if (cudaGetLastError() != cudaSuccess) return ATOM_ERR_CUDA;
+  }
+  return ATOM_OK;
+}
+
+// Co-resident CTA pairs of the GEMM kernel on this device (cached per device).
+atom_status_t gemm_pairs(DeviceState *dev, bool pmode, int *pairs) {
+  using namespace atomk::gemm_cfg;
+  if (!dev->gemm_attr[pmode]) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    const void *fn = pmode ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<true>)
+                           : reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<false>);
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+      return ATOM_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * dev->sm_count, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg) != cudaSuccess || clusters < 1)
+      clusters = dev->sm_count / 2;
+    dev->gemm_clusters[pmode] = clusters;
+    dev->gemm_attr[pmode] = true;
+  }
+  *pairs = dev->gemm_clusters[pmode];
+  return ATOM_OK;
 }
 
 }  // namespace
@@ -265,10 +313,9 @@ atom_status_t atom_w4a4_gemm(const uint8_t *qa4, const int8_t *qa8, const float 
                              const uint8_t *qw4, const int8_t *qw8, const float *sw, void *y,
                              int64_t M, int64_t N, int64_t K, int32_t n_outlier, int32_t group,
                              void *workspace, size_t workspace_bytes, atom_stream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   if (!y && M > 0) return ATOM_ERR_INVALID_ARG;
-  return launch_gemm(qa4, qa8, sa, qw4, qw8, sw, y, nullptr, M, N, K, n_outlier, group, stream);
+  return launch_gemm(qa4, qa8, sa, qw4, qw8, sw, y, nullptr, M, N, K, n_outlier, group, workspace,
+                     workspace_bytes, stream);
 }
 
 atom_status_t atom_w4a4_gemm_partials(const uint8_t *qa4, const int8_t *qa8, const float *sa,
@@ -276,14 +323,17 @@ atom_status_t atom_w4a4_gemm_partials(const uint8_t *qa4, const int8_t *qa8, con
                                       int32_t *partials, void *y, int64_t M, int64_t N, int64_t K,
                                       int32_t n_outlier, int32_t group, atom_stream_t stream) {
   if (!partials && M > 0) return ATOM_ERR_INVALID_ARG;
-  return launch_gemm(qa4, qa8, sa, qw4, qw8, sw, y, partials, M, N, K, n_outlier, group, stream);
+  return launch_gemm(qa4, qa8, sa, qw4, qw8, sw, y, partials, M, N, K, n_outlier, group, nullptr,
+                     0, stream);
 }
 
 size_t atom_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  (void)M;
-  (void)N;
-  (void)K;
-  return 0;
+  if (M <= 0 || N <= 0 || K < 256) return 0;
+  DeviceState *dev = nullptr;
+  int pairs = 0;
+  if (current_device(&dev) != ATOM_OK || gemm_pairs(dev, false, &pairs) != ATOM_OK) return 0;
+  const int splits = gemm_splits(M, N, K, pairs);
+  return splits > 1 ? static_cast<size_t>(splits) * M * N * sizeof(float) : 0;
 }
 
 atom_status_t atom_device_status(int clear) {

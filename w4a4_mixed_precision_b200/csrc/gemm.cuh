@@ -125,8 +125,11 @@ struct GemmParams {
   const float *sw;
   __half *y;           // may be null in partials mode
   int32_t *partials;   // partials mode only
+  float *ws;           // splits > 1: fp32 partial outputs [splits][M][N]
   int M, N, K, G;
   int m_tiles, n_tiles, tiles;   // pair tiles of 256 x 256
+  int splits;                    // K splits per tile (1: no split)
+  int items;                     // tiles * splits
   int sa_by_tma;                 // M % 4 == 0: sa rows are 16-byte aligned for TMA
 };
 
@@ -149,6 +152,17 @@ __device__ __forceinline__ void st_global_v4_if(void *p, uint32_t a, uint32_t b,
       : "memory");
 }
 
+// 8-byte store of an fp32 pair, passed as two f32 operands (the accumulator
+// pairs live in 64-bit registers for the f32x2 arithmetic; handing them over
+// as 32-bit integer operands made the compiler spill the accumulators).
+__device__ __forceinline__ void st_global_f2_if(void *p, float2 v, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %3, 0;\n\t@q st.global.v2.f32 [%0], {%1, %2};\n\t}" ::"l"(
+          p),
+      "f"(v.x), "f"(v.y), "r"(static_cast<uint32_t>(pred))
+      : "memory");
+}
+
 __device__ __forceinline__ void st_global_v2_if(void *p, uint32_t a, uint32_t b, bool pred) {
   asm volatile(
       "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %3, 0;\n\t@q st.global.v2.b32 [%0], {%1, %2};\n\t}" ::"l"(
@@ -157,22 +171,28 @@ __device__ __forceinline__ void st_global_v2_if(void *p, uint32_t a, uint32_t b,
       : "memory");
 }
 
-// Walks one CTA pair's (tile, group) sequence; both CTAs of a pair walk the same one.
+// Walks one CTA pair's (item, group) sequence; both CTAs of a pair walk the
+// same one. An item is one output tile and one of its `splits` K ranges: item
+// i is tile i / splits, split i % splits, groups [split*G/splits,
+// (split+1)*G/splits). The pairs take items round-robin.
 struct TileWalk {
-  int tile, g, m0, n0;
+  int item, g, g_end, split, m0, n0;
   __device__ __forceinline__ void start(const GemmParams &p) {
-    tile = blockIdx.x >> 1;
-    g = 0;
+    item = blockIdx.x >> 1;
     set(p);
   }
   __device__ __forceinline__ void set(const GemmParams &p) {
+    const int tile = item / p.splits;
+    split = item - tile * p.splits;
     m0 = (tile % p.m_tiles) * gemm_cfg::kPairM;
     n0 = (tile / p.m_tiles) * gemm_cfg::BN;
+    g = split * p.G / p.splits;
+    g_end = (split + 1) * p.G / p.splits;
   }
+  __device__ __forceinline__ bool last() const { return g == g_end - 1; }
   __device__ __forceinline__ void next(const GemmParams &p) {
-    if (++g == p.G) {
-      g = 0;
-      tile += gridDim.x >> 1;
+    if (++g == g_end) {
+      item += gridDim.x >> 1;
       set(p);
     }
   }
@@ -193,8 +213,16 @@ struct RingPos {
 
 __device__ __forceinline__ int64_t pair_iterations(const GemmParams &p) {
   const int pair = static_cast<int>(blockIdx.x >> 1), pairs = static_cast<int>(gridDim.x >> 1);
-  const int mine = p.tiles > pair ? (p.tiles - pair + pairs - 1) / pairs : 0;
-  return static_cast<int64_t>(mine) * p.G;
+  if (p.splits == 1) {
+    const int mine = p.items > pair ? (p.items - pair + pairs - 1) / pairs : 0;
+    return static_cast<int64_t>(mine) * p.G;
+  }
+  int64_t n = 0;
+  for (int it = pair; it < p.items; it += pairs) {
+    const int s = it % p.splits;
+    n += (s + 1) * p.G / p.splits - s * p.G / p.splits;
+  }
+  return n;
 }
 
 // ------------------------------------------------------------------ unpack role
@@ -455,18 +483,27 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         mbar_arrive(&sempty[sl]);
       }
 
-      if (w.g == p.G - 1) {
-        // epilogue: this thread's 128 columns of its row, 8 per 16-byte store
+      if (w.last()) {
+        // epilogue: this thread's 128 columns of its row, 8 per step: fp16 Y,
+        // or, when K is split, this split's fp32 partial tile. One loop with
+        // both (predicated) stores: two separately unrolled loops over the
+        // accumulators made the compiler spill them.
         const int row = w.m0 + BM * rank + lrow;
-        const bool have_y = p.y != nullptr;
+        const bool to_y = p.splits == 1 && p.y != nullptr, to_ws = p.splits > 1;
+        __half *y_row = p.y + static_cast<int64_t>(row < p.M ? row : 0) * p.N;
+        float *ws_row = p.ws + (static_cast<int64_t>(w.split) * p.M + (row < p.M ? row : 0)) * p.N;
 #pragma unroll
         for (int v = 0; v < 16; ++v) {
           const int col = w.n0 + kHalfN * hh + 8 * v;
           const float2 *a = acc + 4 * v;
-          const bool oky = have_y && row < p.M && col < p.N;
-          st_global_v4_if(p.y + static_cast<int64_t>(oky ? row : 0) * p.N + (oky ? col : 0),
-                          pack_half2_rn(a[0].x, a[0].y), pack_half2_rn(a[1].x, a[1].y),
-                          pack_half2_rn(a[2].x, a[2].y), pack_half2_rn(a[3].x, a[3].y), oky);
+          const bool in = row < p.M && col < p.N;
+          const int cc = in ? col : 0;
+          st_global_v4_if(y_row + cc, pack_half2_rn(a[0].x, a[0].y), pack_half2_rn(a[1].x, a[1].y),
+                          pack_half2_rn(a[2].x, a[2].y), pack_half2_rn(a[3].x, a[3].y),
+                          in && to_y);
+          // fp32 partials go out as 8-byte stores of the accumulator pairs
+#pragma unroll
+          for (int k = 0; k < 4; ++k) st_global_f2_if(ws_row + cc + 2 * k, a[k], in && to_ws);
         }
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
@@ -617,6 +654,31 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   if (warp == 0) {
     tc_fence_after_sync();
     tmem_dealloc_pair(tbase, kTmemCols);
+  }
+}
+
+// Sums the fp32 partial tiles of a split GEMM in split order and writes fp16
+// Y: thread t handles columns [8t, 8t + 8) of the flattened [M][N] output
+// (N % 8 == 0).
+__global__ void __launch_bounds__(256)
+splitk_reduce_kernel(const float *__restrict__ ws, __half *__restrict__ y, int64_t count8,
+                     int64_t mn, int splits) {
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < count8;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float4 a = __ldg(reinterpret_cast<const float4 *>(ws) + 2 * t);
+    float4 b = __ldg(reinterpret_cast<const float4 *>(ws) + 2 * t + 1);
+    for (int s = 1; s < splits; ++s) {
+      const float4 *src = reinterpret_cast<const float4 *>(ws + s * mn) + 2 * t;
+      const float4 c = __ldg(src), d = __ldg(src + 1);
+      a.x += c.x; a.y += c.y; a.z += c.z; a.w += c.w;
+      b.x += d.x; b.y += d.y; b.z += d.z; b.w += d.w;
+    }
+    uint4 o;
+    o.x = pack_half2_rn(a.x, a.y);
+    o.y = pack_half2_rn(a.z, a.w);
+    o.z = pack_half2_rn(b.x, b.y);
+    o.w = pack_half2_rn(b.z, b.w);
+    reinterpret_cast<uint4 *>(y)[t] = o;
   }
 }
 
