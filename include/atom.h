@@ -162,6 +162,34 @@ ATOM_API atom_status_t atom_w4a4_gemm_partials(const uint8_t *qa4, const int8_t 
 ATOM_API size_t atom_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
+ * atom_w4a4_gemm_noalloc -- atom_w4a4_gemm for callers that cannot allocate
+ * device memory around the call: code running while a CUDA graph is captured,
+ * serving runtimes that give all device memory to a fixed pool at start-up, C
+ * callers with no device allocator. (The pages describe no such entry point;
+ * it is a deployment convenience of this library.)
+ *
+ * Arguments, layouts, result and errors are those of atom_w4a4_gemm without
+ * the workspace. When the shape splits K (small M), the split's fp32 partial
+ * tiles go to a fixed 8 MiB array in the library's device memory instead of a
+ * caller workspace; every GPU that loads the library holds that array until
+ * the process exits. A shape whose partials would need more than 8 MiB
+ * (splits * M * N * 4 bytes, see atom_gemm_workspace_bytes) returns
+ * ATOM_ERR_SHAPE before anything is launched. The call allocates nothing.
+ *
+ * All calls on a device share the array, and a call leaves its partials in
+ * it: two calls that overlap on the GPU (other streams, other host threads)
+ * race and must be ordered by the caller. The first call on each device does
+ * a one-time set-up (it looks up the array's device address and the kernel's
+ * launch limits) and should come before any stream capture.
+ */
+ATOM_API atom_status_t atom_w4a4_gemm_noalloc(const uint8_t *qa4, const int8_t *qa8,
+                                              const float *sa, const uint8_t *qw4,
+                                              const int8_t *qw8, const float *sw, void *y,
+                                              int64_t M, int64_t N, int64_t K,
+                                              int32_t n_outlier, int32_t group,
+                                              atom_stream_t stream);
+
+/*
  * atom_device_status -- first device-detected error since the last clear on the
  * current device (ATOM_OK if none). Synchronises the current device. With
  * clear != 0 the status is reset to ATOM_OK afterwards.

@@ -49,6 +49,8 @@ SIGNATURES = {
                                                      ct.c_int32, ct.c_int32, ct.c_void_p],
                                 ct.c_int),
     "atom_gemm_workspace_bytes": ([ct.c_int64, ct.c_int64, ct.c_int64], ct.c_size_t),
+    "atom_w4a4_gemm_noalloc": ([ct.c_void_p] * 7 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_int32,
+                                                    ct.c_int32, ct.c_void_p], ct.c_int),
     "atom_device_status": ([ct.c_int], ct.c_int),
     "atom_status_string": ([ct.c_int], ct.c_char_p),
     "atom_version": ([], ct.c_int),
@@ -175,6 +177,23 @@ def atom_w4a4_gemm(qa: Quantized, qw: Quantized, K: int, y: Optional[torch.Tenso
         _dev(qw.q8, torch.int8, "qw8"), _dev(qw.scales, torch.float32, "sw"),
         _dev(y, torch.float16, "y"), M, N, K, N_OUTLIER, GROUP, ws_ptr, ws_bytes, _stream(stream))
     _check("atom_w4a4_gemm", st)
+    return y
+
+
+def atom_w4a4_gemm_noalloc(qa: Quantized, qw: Quantized, K: int,
+                           y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """atom_w4a4_gemm for callers that cannot allocate around the call: a split
+    of K keeps its partials in the library's fixed 8 MiB device array (see
+    include/atom.h). Pass `y` to keep this wrapper allocation-free as well."""
+    M, N = qa.rows, qw.rows
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=qa.q4.device)
+    st = lib().atom_w4a4_gemm_noalloc(
+        _dev(qa.q4, torch.uint8, "qa4"), _dev(qa.q8, torch.int8, "qa8"),
+        _dev(qa.scales, torch.float32, "sa"), _dev(qw.q4, torch.uint8, "qw4"),
+        _dev(qw.q8, torch.int8, "qw8"), _dev(qw.scales, torch.float32, "sw"),
+        _dev(y, torch.float16, "y"), M, N, K, N_OUTLIER, GROUP, _stream(stream))
+    _check("atom_w4a4_gemm_noalloc", st)
     return y
 
 

@@ -25,6 +25,7 @@ struct DeviceState {
   uint32_t quant_smem_set = 0;
   uint32_t quant_occ_smem = 0;  // shared-memory size the cached occupancy is for
   int quant_occ = 0;            // co-resident quantizer CTAs per SM at that size
+  void *noalloc_scratch = nullptr;  // device address of g_noalloc_scratch on this device
 };
 
 DeviceState g_devices[kMaxDevices];
@@ -365,3 +366,62 @@ const char *atom_status_string(atom_status_t status) {
 int atom_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free GEMM
+//
+// Some callers cannot allocate device memory around a GEMM call: code that
+// runs while a CUDA graph is being captured (an allocation there is not part
+// of the graph and breaks replay), serving runtimes that hand every byte of
+// device memory to a fixed pool at start-up, and C callers with no device
+// allocator of their own. atom_w4a4_gemm needs scratch only when it splits K
+// (small M), and takes it from the caller. This entry point takes it instead
+// from a fixed array in the library's device memory.
+
+namespace {
+
+// Scratch of atom_w4a4_gemm_noalloc: the fp32 partial tiles of a split-K call,
+// splits * M * N floats. Every GPU that loads the library holds it until exit.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB
+__device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of the scratch on the current device. In host code the name
+// g_noalloc_scratch is a host-side stand-in, not a device address, so the
+// address is looked up once per device, with that device current.
+atom_status_t noalloc_scratch(DeviceState *dev, void **out) {
+  if (dev->noalloc_scratch == nullptr) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (dev->noalloc_scratch == nullptr) {
+      void *p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return ATOM_ERR_CUDA;
+      dev->noalloc_scratch = p;
+    }
+  }
+  *out = dev->noalloc_scratch;
+  return ATOM_OK;
+}
+
+}  // namespace
+
+extern "C" ATOM_API atom_status_t atom_w4a4_gemm_noalloc(
+    const uint8_t *qa4, const int8_t *qa8, const float *sa, const uint8_t *qw4, const int8_t *qw8,
+    const float *sw, void *y, int64_t M, int64_t N, int64_t K, int32_t n_outlier, int32_t group,
+    atom_stream_t stream) {
+  if (M < 0 || N < 0) return ATOM_ERR_INVALID_ARG;
+  atom_status_t st = check_method_params(K, n_outlier, group);
+  if (st != ATOM_OK) return st;
+  if (M == 0) return ATOM_OK;
+  if (!y) return ATOM_ERR_INVALID_ARG;
+  DeviceState *dev = nullptr;
+  if ((st = current_device(&dev)) != ATOM_OK) return st;
+  int pairs = 0;
+  if ((st = gemm_pairs(dev, false, &pairs)) != ATOM_OK) return st;
+  const int splits = gemm_splits(M, N, K, pairs);
+  if (splits > 1 &&
+      static_cast<double>(splits) * M * N * sizeof(float) > static_cast<double>(kNoAllocScratchBytes))
+    return ATOM_ERR_SHAPE;   // the split's partial tiles do not fit in the fixed scratch
+  void *scratch = nullptr;
+  if ((st = noalloc_scratch(dev, &scratch)) != ATOM_OK) return st;
+  return launch_gemm(qa4, qa8, sa, qw4, qw8, sw, y, nullptr, M, N, K, n_outlier, group, scratch,
+                     kNoAllocScratchBytes, stream);
+}
