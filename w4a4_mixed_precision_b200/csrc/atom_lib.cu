@@ -210,6 +210,13 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
       !encode_2d(&maps.w8, u8, qw8, 128, N, 128, 128, BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&maps.sw, f32, sw, N, G, N * 4, BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
     return ATOM_ERR_CUDA;
+  if (y) {
+    if (!encode_2d(&maps.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, y, N, M, N * 2, 64, 32,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return ATOM_ERR_CUDA;
+  } else {
+    maps.y = maps.sw;   // not used by the kernel
+  }
   if (sa_by_tma) {
     if (!encode_2d(&maps.sa, f32, sa, M, G, M * 4, BM, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
       return ATOM_ERR_CUDA;

@@ -30,6 +30,7 @@
 //                 int8 A and W tiles. Freed by the MMA's commit.
 //   scale ring    (unpackers -> drain): sa and sw laid out for the drain's
 //                 TMEM fragments. Freed by the drain.
+// plus one 4 KB Y staging box per drain warp (drain -> TMA store).
 // Roles in each CTA:
 //
 //   producer (warp 0, lane 0)  TMA copies into the packed ring.
@@ -48,7 +49,8 @@
 //                      per load, accumulates sa*sw*P into 128 fp32 registers,
 //                      and arrives on the leader's "accumulator free" barrier
 //                      once its loads are done. After the last group of a
-//                      tile: fp16 stores.
+//                      tile: fp16 Y, staged per warp in shared memory as two
+//                      32x64 boxes and written by TMA tensor stores.
 //
 // Exact integer -> float without a conversion instruction: every accumulator
 // starts at the int32 0x4B400000 (the bits of C = 1.5*2^23) and the MMAs add
@@ -80,7 +82,7 @@ constexpr int kPairM = 2 * BM;
 constexpr int kThreads = 512;
 constexpr int kUnpackThreads = 192;  // warps 2..7
 constexpr int kUnpackWarps = kUnpackThreads / 32;
-constexpr int kNP = 6;           // packed ring slots
+constexpr int kNP = 4;           // packed ring slots
 constexpr int kNU = 3;           // operand ring slots
 constexpr int kNS = 6;           // scale ring slots
 // packed slot: INT4 A at 0, INT4 W at kPackWOff; or one INT8 tile at 0
@@ -100,7 +102,10 @@ constexpr uint32_t kBarBytes = 1024;
 constexpr uint32_t kUOff = kBarBytes;                    // from the 1024-aligned base
 constexpr uint32_t kPOff = kUOff + kNU * kUSlot;
 constexpr uint32_t kSOff = kPOff + kNP * kPSlot;
-constexpr uint32_t kSmemBytes = kSOff + kNS * kSSlot + 1024;  // + alignment slack
+// Y staging: one 32-row x 64-column fp16 box (128-byte swizzle) per drain warp
+constexpr uint32_t kYSlot = 32 * 128;
+constexpr uint32_t kYOff = (kSOff + kNS * kSSlot + 1023u) & ~1023u;
+constexpr uint32_t kSmemBytes = kYOff + 8 * kYSlot + 1024;  // + alignment slack
 constexpr int kPackedChunks = (BM + BW) * 4;                    // 16-B chunks per INT4 group
 constexpr int kChunksPerThread = (kPackedChunks + kUnpackThreads - 1) / kUnpackThreads;
 constexpr int kInt8Chunks = (kABytes + kBBytes) / 16;           // 16-B chunks of an INT8 group
@@ -115,6 +120,7 @@ static_assert(kABytes <= kSwLinOff && kBBytes <= kSwLinOff, "INT8 tile must fit 
 static_assert(kPSlot % 1024 == 0 && kUSlot % 1024 == 0, "slots must keep 1024-byte alignment");
 static_assert(kSOff % 16 == 0 && kSSlot % 16 == 0, "scale slots must be 16-byte aligned");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kYOff % 1024 == 0 && kYSlot % 1024 == 0, "Y staging must keep 1024-byte alignment");
 static_assert(2 * 128 * (kUnpackRegs + kDrainRegs) == 65536, "register split must fill the file");
 }  // namespace gemm_cfg
 
@@ -308,6 +314,7 @@ struct GemmMaps {
   CUtensorMap w8;   // INT8 W: [N][128], boxes 128 x 128 bytes, 128-byte swizzle
   CUtensorMap sa;   // fp32 [G][M], boxes of 1 x 128 (used when M % 4 == 0)
   CUtensorMap sw;   // fp32 [G][N], boxes of 1 x 256
+  CUtensorMap y;    // fp16 Y [M][N], boxes of 32 rows x 64 columns, 128-byte swizzle (stores)
 };
 
 // Hardware barrier ids for the role-internal gathers (0 is __syncthreads).
@@ -333,6 +340,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   uint8_t *uring = smem + kUOff;
   uint8_t *pring = smem + kPOff;
   uint8_t *sring = smem + kSOff;
+  uint8_t *ystage = smem + kYOff;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = static_cast<int>(cluster_cta_rank());
@@ -484,31 +492,50 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       }
 
       if (w.last()) {
-        // epilogue: this thread's 128 columns of its row, 8 per step: fp16 Y,
-        // or, when K is split, this split's fp32 partial tile. One loop with
-        // both (predicated) stores: two separately unrolled loops over the
-        // accumulators made the compiler spill them.
-        const int row = w.m0 + BM * rank + lrow;
+        // epilogue, 8 columns of this thread's row per step. fp16 Y goes out
+        // through shared memory and the TMA, 64 columns at a time: each thread
+        // writes its row of the warp's 32 x 64 box (128-byte swizzle: 16-byte
+        // chunk j of row r sits at chunk j ^ (r & 7)), then one lane stores
+        // the box (the rows and columns past M and N are not written). When K
+        // is split, this split's fp32 partial tile goes out instead, as
+        // predicated 8-byte stores. One loop without branches around the
+        // accumulator reads: the compiler spills them otherwise.
         const bool to_y = p.splits == 1 && p.y != nullptr, to_ws = p.splits > 1;
-        __half *y_row = p.y + static_cast<int64_t>(row < p.M ? row : 0) * p.N;
+        const int row = w.m0 + BM * rank + lrow;
+        const int row0 = w.m0 + BM * rank + 32 * q;   // the warp's first row
         float *ws_row = p.ws + (static_cast<int64_t>(w.split) * p.M + (row < p.M ? row : 0)) * p.N;
+        uint8_t *ybuf = ystage + dw * kYSlot;
 #pragma unroll
         for (int v = 0; v < 16; ++v) {
+          if ((v & 7) == 0) {
+            if (lane == 0) bulk_wait_group_read0();   // the previous box has left the buffer
+            __syncwarp();
+          }
           const int col = w.n0 + kHalfN * hh + 8 * v;
           const float2 *a = acc + 4 * v;
           const bool in = row < p.M && col < p.N;
           const int cc = in ? col : 0;
-          st_global_v4_if(y_row + cc, pack_half2_rn(a[0].x, a[0].y), pack_half2_rn(a[1].x, a[1].y),
-                          pack_half2_rn(a[2].x, a[2].y), pack_half2_rn(a[3].x, a[3].y),
-                          in && to_y);
-          // fp32 partials go out as 8-byte stores of the accumulator pairs
+          st_shared_v4(ybuf + lane * 128 + (((v & 7) ^ (lane & 7)) << 4),
+                       pack_half2_rn(a[0].x, a[0].y), pack_half2_rn(a[1].x, a[1].y),
+                       pack_half2_rn(a[2].x, a[2].y), pack_half2_rn(a[3].x, a[3].y));
 #pragma unroll
           for (int k = 0; k < 4; ++k) st_global_f2_if(ws_row + cc + 2 * k, a[k], in && to_ws);
+          if ((v & 7) == 7) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            const int col0 = w.n0 + kHalfN * hh + 64 * (v >> 3);
+            if (lane == 0 && to_y && row0 < p.M && col0 < p.N) {
+              tma_store_2d(&maps.y, ybuf, col0, row0);
+              bulk_commit_group();
+            }
+          }
         }
 #pragma unroll
         for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
       }
     }
+    // the Y boxes must be out of shared memory before the CTA exits
+    if (lane == 0) bulk_wait_group0();
   } else {
     regs_decrease<kUnpackRegs>();
     if (warp == 0) {
