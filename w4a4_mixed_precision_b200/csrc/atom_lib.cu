@@ -23,8 +23,9 @@ struct DeviceState {
   bool gemm_attr[2] = {false, false};
   int gemm_clusters[2] = {0, 0};  // co-resident CTA pairs of the GEMM kernel
   uint32_t quant_smem_set = 0;
-  uint32_t quant_occ_smem = 0;  // shared-memory size the cached occupancy is for
-  int quant_occ = 0;            // co-resident quantizer CTAs per SM at that size
+  int64_t quant_k = -1;         // K the cached quantizer launch shape is for
+  int quant_stages = 0;         // rows in flight per CTA for that K
+  int quant_occ = 0;            // co-resident quantizer CTAs per SM for that K
   void *noalloc_scratch = nullptr;  // device address of g_noalloc_scratch on this device
 };
 
@@ -80,33 +81,46 @@ atom_status_t launch_quant(const void *x, int64_t rows, int64_t K, int64_t ld,
   DeviceState *dev = nullptr;
   if ((st = current_device(&dev)) != ATOM_OK) return st;
 
-  int stages = 3;
-  atomk::QuantLayout L = atomk::quant_layout(static_cast<int>(K), stages);
-  if (L.total > 110u * 1024u) {
-    stages = 2;
-    L = atomk::quant_layout(static_cast<int>(K), stages);
-  }
-  if (static_cast<int>(L.total) > dev->smem_optin) return ATOM_ERR_SHAPE;
-  if (dev->quant_smem_set < L.total) {
+  // Rows in flight per CTA (2 or 3): the choice that keeps the most rows in
+  // flight per SM, and at a tie the one with more CTAs (worked out once per K
+  // and cached).
+  int stages = 0, occ = 0;
+  {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (cudaFuncSetAttribute(atomk::reorder_quant_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(L.total)) != cudaSuccess)
-      return ATOM_ERR_CUDA;
-    dev->quant_smem_set = L.total;
+    if (dev->quant_k != K) {
+      int best_stages = 0, best_occ = 0;
+      for (int n = 3; n >= 2; --n) {
+        const atomk::QuantLayout l = atomk::quant_layout(static_cast<int>(K), n);
+        if (static_cast<int>(l.total) > dev->smem_optin) continue;
+        if (dev->quant_smem_set < l.total) {
+          if (cudaFuncSetAttribute(atomk::reorder_quant_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(l.total)) != cudaSuccess)
+            return ATOM_ERR_CUDA;
+          dev->quant_smem_set = l.total;
+        }
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, atomk::reorder_quant_kernel,
+                                                          atomk::kQuantThreads,
+                                                          l.total) != cudaSuccess)
+          return ATOM_ERR_CUDA;
+        // most rows in flight per SM; at a tie, more CTAs (more warps)
+        if (per_sm * n > best_occ * best_stages ||
+            (per_sm * n == best_occ * best_stages && per_sm > best_occ)) {
+          best_occ = per_sm;
+          best_stages = n;
+        }
+      }
+      if (best_stages == 0) return ATOM_ERR_SHAPE;
+      dev->quant_stages = best_stages;
+      dev->quant_occ = best_occ;
+      dev->quant_k = K;
+    }
+    stages = dev->quant_stages;
+    occ = dev->quant_occ;
   }
-  // One persistent wave: as many CTAs as fit on the device at once.
-  if (dev->quant_occ_smem != L.total) {
-    std::lock_guard<std::mutex> lock(g_mutex);
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, atomk::reorder_quant_kernel,
-                                                      atomk::kQuantThreads,
-                                                      L.total) != cudaSuccess)
-      return ATOM_ERR_CUDA;
-    dev->quant_occ = per_sm < 1 ? 1 : per_sm;
-    dev->quant_occ_smem = L.total;
-  }
-  const int64_t want = static_cast<int64_t>(dev->quant_occ) * dev->sm_count;
+  const atomk::QuantLayout L = atomk::quant_layout(static_cast<int>(K), stages);
+  const int64_t want = static_cast<int64_t>(occ) * dev->sm_count;
   const int grid = static_cast<int>(rows < want ? rows : want);
   atomk::reorder_quant_kernel<<<grid, atomk::kQuantThreads, L.total,
                                 reinterpret_cast<cudaStream_t>(stream)>>>(

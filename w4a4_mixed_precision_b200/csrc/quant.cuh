@@ -12,8 +12,9 @@
 //  * each CTA is persistent over rows r = blockIdx.x + i*gridDim.x; a whole
 //    fp16 row is brought into shared memory by one bulk copy (TMA engine,
 //    mbarrier completion), up to kQuantMaxStages rows in flight per CTA; each
-//    warp frees a stage through its own arrival on an "empty" mbarrier, so the
-//    warps of a CTA never wait for one another while the ring has room;
+//    quantizing warp frees a stage through its own arrival on an "empty"
+//    mbarrier, and a ninth warp issues the copy that refills it, so the
+//    quantizing warps never wait for one another while the ring has room;
 //  * at start-up each CTA turns the outlier list into a gather table in shared
 //    memory (uint16 [K]): for every group and lane, the byte offsets inside a
 //    staged row of the 16 channels that lane quantizes, in the lane's gather
@@ -36,8 +37,8 @@
 
 namespace atomk {
 
-constexpr int kQuantThreads = 256;
-constexpr int kQuantWarps = kQuantThreads / 32;
+constexpr int kQuantWarps = 8;                          // quantizing warps
+constexpr int kQuantThreads = 32 * (kQuantWarps + 1);     // + one copy-issuing warp
 constexpr int kQuantMaxStages = 4;
 // Gather-table entries are 16-bit byte offsets into a staged fp16 row.
 constexpr int kQuantMaxK = 32768;
@@ -175,6 +176,41 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     return;
   }
 
+  if (warp == kQuantWarps) {
+    // ---- copy issuer: refills each stage slot as soon as all quantizing
+    // warps have released it (slot i % stages_n holds row blockIdx.x + i*grid;
+    // rows 0..stages_n-1 were issued above).
+    if (lane == 0) {
+      int sl = 0;
+      uint32_t eph = 0;
+      int64_t i = stages_n;
+      for (;; ++i) {
+        const int64_t r = blockIdx.x + i * grid;
+        if (r >= rows) break;
+        if (!mbar_wait(&empty[sl], eph, &flags[1])) {
+          if (!flags[1]) report_status(6 /* ATOM_ERR_TIMEOUT */);
+          flags[1] = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[sl], L.row_bytes);
+        bulk_load(stage_base + sl * L.row_bytes, x + r * ld, L.row_bytes, &full[sl]);
+        if (++sl == stages_n) {
+          sl = 0;
+          eph ^= 1u;
+        }
+      }
+      if (flags[1]) {
+        // after an abort, give the copies that may still be in flight (the
+        // last one issued into each slot) a bounded chance to land before the
+        // CTA's shared memory is released
+        for (int64_t j = (i > stages_n ? i - stages_n : 0); j < i; ++j)
+          if (blockIdx.x + j * grid < rows)
+            (void)mbar_wait(&full[j % stages_n], static_cast<uint32_t>((j / stages_n) & 1), nullptr);
+      }
+    }
+    return;
+  }
+
   // ---- per-lane constants: group g = pass*32 + 4*warp + team, elements
   // [16*sub, 16*sub + 16) of the group.
   const int sub = lane & 7;
@@ -189,11 +225,10 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     sel_hi |= static_cast<uint32_t>((j + 4 - krot) & 7) << (4 * j);
   }
 
-  int64_t done = 0;  // rows this CTA has finished
-  // Stage slot and barrier parity of row i and of row i-1, advanced by
-  // counting (no division on the per-row path).
-  int s = 0, s_prev = 0;
-  uint32_t ph = 0, ph_prev = 0;
+  // Stage slot and barrier parity of row i, advanced by counting (no
+  // division on the per-row path).
+  int s = 0;
+  uint32_t ph = 0;
   for (int64_t i = 0;; ++i) {
     const int64_t r = blockIdx.x + i * grid;
     if (r >= rows) break;
@@ -266,36 +301,10 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
 
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-    done = i + 1;
-
-    // Refill the stage of the previous row: one row of slack, so the issuing
-    // thread rarely waits for the slowest warp.
-    if (tid == 0 && i >= 1) {
-      const int64_t nr = blockIdx.x + (i - 1 + stages_n) * grid;
-      if (nr < rows) {
-        if (!mbar_wait(&empty[s_prev], ph_prev, &flags[1])) {
-          report_status(6 /* ATOM_ERR_TIMEOUT */);
-          flags[1] = 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&full[s_prev], L.row_bytes);
-        bulk_load(stage_base + s_prev * L.row_bytes, x + nr * ld, L.row_bytes, &full[s_prev]);
-      }
-    }
-    s_prev = s;
-    ph_prev = ph;
     if (++s == stages_n) {
       s = 0;
       ph ^= 1u;
     }
-  }
-
-  // After an abort, give the copies still in flight a bounded chance to land
-  // before the CTA's shared memory is released.
-  if (tid == 0 && flags[1]) {
-    for (int64_t j = done; j < done + stages_n; ++j)
-      if (blockIdx.x + j * grid < rows)
-        (void)mbar_wait(&full[j % stages_n], static_cast<uint32_t>((j / stages_n) & 1), nullptr);
   }
 }
 
