@@ -174,6 +174,8 @@ def main():
                     help="seconds of CPU oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cublas", action="store_true",
+                    help="skip the fp16 cuBLAS GEMM of the same shape reported beside the result")
     ap.add_argument("--m", type=int, default=None,
                     help="use only the first M activation rows (small profiling cases)")
     args = ap.parse_args()
@@ -302,6 +304,29 @@ def main():
                "d2h_bytes_per_step": w.M * w.N * 2, "ms_per_step": round(e2e_ms, 4),
                "steps": e2e_steps}
 
+    # -------- fp16 cuBLAS GEMM of the same shape (torch.matmul), a library baseline
+    cublas = None
+    if not args.no_cublas:
+        W16 = torch.from_numpy(W_h.view(np.uint16)).to(dev).view(torch.float16)
+        y16 = torch.empty((w.M, w.N), dtype=torch.float16, device=dev)
+        for _ in range(3):
+            torch.matmul(A, W16.t(), out=y16)
+        torch.cuda.synchronize()
+        n_cb = max(3, min(20, n_steps // 10))
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(n_cb):
+            torch.matmul(A, W16.t(), out=y16)
+        c1.record(stream)
+        torch.cuda.synchronize()
+        cb_ms = c0.elapsed_time(c1) / n_cb
+        cublas = {"value": round(2.0 * w.M * w.N * w.K / (cb_ms * 1e-3) / 1e12, 2),
+                  "unit": "TFLOP/s", "ms": round(cb_ms, 4), "steps": n_cb,
+                  "kind": "torch.matmul fp16 x fp16 -> fp16 (cuBLAS), same M, N, K, "
+                          "operands resident in HBM"}
+        del W16, y16
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -367,6 +392,9 @@ def main():
         "gpu_launches": 2 * n_steps,
         "e2e": e2e,
     }
+    if cublas is not None:
+        cublas["w4a4_gemm_speedup"] = round(cublas["ms"] / gemm_avg, 3)
+        line["fp16_cublas"] = cublas
     if world == 1 and not args.no_cpu_baseline:
         ops_s, rows, dt, cores = cpu_oracle_run(w, A_h, W_h, idx_h, args.cpu_budget)
         line["cpu_baseline"] = {"value": round(ops_s / 1e12, 6), "unit": "TOPS", "cores": cores,

@@ -190,6 +190,35 @@ ATOM_API atom_status_t atom_w4a4_gemm_noalloc(const uint8_t *qa4, const int8_t *
                                               atom_stream_t stream);
 
 /*
+ * atom_w8a8_gemm -- the 8-bit comparator of the W4A4 GEMM: INT8 activations
+ * and weights with one scale per activation row and one per weight row,
+ *
+ *   y[m][n] = fp16( float(P) * (sa[m] * sw[n]) ),  P = sum_k qa[m][k] * qw[n][k]
+ *
+ * where P is the exact int32 dot product over all of K (no groups; a
+ * per-tensor scale is constant sa and sw). Source: the Atom paper's comparison
+ * of its W4A4 kernels with 8-bit weight-and-activation serving
+ * ("Atom: Low-bit Quantization for Efficient and Accurate LLM Serving",
+ * summary of results); the pages give no INT8 kernel, so this restates the
+ * plain per-row x per-column scaled INT8 GEMM on the same tensor-core pipeline
+ * as the W4A4 GEMM.
+ *
+ *   qa  int8 [M][K] device, row-major (row pitch K bytes).
+ *   sa  fp32 [M] device.
+ *   qw  int8 [N][K] device, row-major.
+ *   sw  fp32 [N] device.
+ *   y   fp16 [M][N] device (output), row-major, written in full.
+ * Preconditions (else ATOM_ERR_SHAPE before any launch): K % 16 == 0,
+ * 16 <= K <= 131072 (the int32 sum cannot overflow), N % 8 == 0. M = 0 or
+ * N = 0 is a no-op. qa, qw, y and sw must be 16-byte aligned, sa 4-byte
+ * (else ATOM_ERR_ALIGN). Stream-ordered, allocates nothing; the result is
+ * deterministic.
+ */
+ATOM_API atom_status_t atom_w8a8_gemm(const int8_t *qa, const float *sa, const int8_t *qw,
+                                      const float *sw, void *y, int64_t M, int64_t N,
+                                      int64_t K, atom_stream_t stream);
+
+/*
  * atom_device_status -- first device-detected error since the last clear on the
  * current device (ATOM_OK if none). Synchronises the current device. With
  * clear != 0 the status is reset to ATOM_OK afterwards.

@@ -22,8 +22,11 @@ def partials(qa: np.ndarray, qw: np.ndarray) -> np.ndarray:
     qw = np.asarray(qw)
     if qa.dtype != np.int8 or qw.dtype != np.int8 or qa.shape[1] != qw.shape[1]:
         raise ValueError("qa [M, K] and qw [N, K] must be int8 with the same K")
-    P = qa.astype(np.float64) @ qw.astype(np.float64).T
-    return np.rint(P).astype(np.int64)
+    a = qa.astype(np.float64)
+    P = np.empty((qa.shape[0], qw.shape[0]), dtype=np.int64)
+    for n0 in range(0, qw.shape[0], 2048):   # blocks of W rows bound the float64 copy
+        P[:, n0:n0 + 2048] = np.rint(a @ qw[n0:n0 + 2048].astype(np.float64).T)
+    return P
 
 
 def output64(qa: np.ndarray, sa: np.ndarray, qw: np.ndarray, sw: np.ndarray) -> np.ndarray:

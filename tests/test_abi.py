@@ -117,3 +117,23 @@ def test_python_binding_refuses_cpu_tensors(lib):
     idx = torch.arange(128, dtype=torch.int32)
     with pytest.raises(ValueError):
         atom.atom_reorder_quant(x, idx)
+
+
+def w8a8(lib, qa=A16, sa=A16, qw=A16, sw=A16, y=A16, M=256, N=256, K=256):
+    return lib.atom_w8a8_gemm(qa, sa, qw, sw, y, M, N, K, None)
+
+
+def test_w8a8_checks_arguments_on_the_host(lib):
+    assert w8a8(lib, M=0) == OK
+    assert w8a8(lib, N=0) == OK
+    assert w8a8(lib, M=-1) == INVALID
+    assert w8a8(lib, K=8) == SHAPE          # K below 16
+    assert w8a8(lib, K=264) == SHAPE        # K % 16 != 0
+    assert w8a8(lib, K=131072 + 16) == SHAPE   # the int32 sum could overflow
+    assert w8a8(lib, N=260) == SHAPE        # N % 8 != 0
+    assert w8a8(lib, qa=0) == INVALID
+    assert w8a8(lib, y=0) == INVALID
+    assert w8a8(lib, qa=MIS) == ALIGN
+    assert w8a8(lib, qw=A16 + 8) == ALIGN
+    assert w8a8(lib, sw=A16 + 4) == ALIGN   # sw is read as 16-byte vectors
+    assert w8a8(lib, sa=MIS) == ALIGN

@@ -51,6 +51,8 @@ SIGNATURES = {
     "atom_gemm_workspace_bytes": ([ct.c_int64, ct.c_int64, ct.c_int64], ct.c_size_t),
     "atom_w4a4_gemm_noalloc": ([ct.c_void_p] * 7 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_int32,
                                                     ct.c_int32, ct.c_void_p], ct.c_int),
+    "atom_w8a8_gemm": ([ct.c_void_p] * 5 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_void_p],
+                       ct.c_int),
     "atom_device_status": ([ct.c_int], ct.c_int),
     "atom_status_string": ([ct.c_int], ct.c_char_p),
     "atom_version": ([], ct.c_int),
@@ -217,6 +219,23 @@ def atom_w4a4_gemm_partials(qa: Quantized, qw: Quantized, K: int,
         M, N, K, N_OUTLIER, GROUP, _stream(stream))
     _check("atom_w4a4_gemm_partials", st)
     return partials, y
+
+
+def atom_w8a8_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,
+                   y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """W8A8 comparator: y = fp16(float(qa @ qw^T) * sa[:, None] * sw[None, :]) with int8
+    qa [M, K], qw [N, K] and fp32 scales sa [M], sw [N] (see include/atom.h)."""
+    M, K = qa.shape
+    N = qw.shape[0]
+    if qw.shape[1] != K or sa.shape != (M,) or sw.shape != (N,):
+        raise ValueError("atom_w8a8_gemm: shapes must be qa [M, K], qw [N, K], sa [M], sw [N]")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=qa.device)
+    st = lib().atom_w8a8_gemm(
+        _dev(qa, torch.int8, "qa"), _dev(sa, torch.float32, "sa"), _dev(qw, torch.int8, "qw"),
+        _dev(sw, torch.float32, "sw"), _dev(y, torch.float16, "y"), M, N, K, _stream(stream))
+    _check("atom_w8a8_gemm", st)
+    return y
 
 
 def atom_gemm_workspace_bytes(M: int, N: int, K: int) -> int:

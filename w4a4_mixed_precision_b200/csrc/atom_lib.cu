@@ -9,6 +9,7 @@
 #include "gemm.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
+#include "w8a8.cuh"
 
 namespace {
 
@@ -22,6 +23,8 @@ struct DeviceState {
   int smem_optin = 0;
   bool gemm_attr[2] = {false, false};
   int gemm_clusters[2] = {0, 0};  // co-resident CTA pairs of the GEMM kernel
+  bool w8a8_attr = false;
+  int w8a8_clusters = 0;          // co-resident CTA pairs of the W8A8 kernel
   uint32_t quant_smem_set = 0;
   int64_t quant_k = -1;         // K the cached quantizer launch shape is for
   int quant_stages = 0;         // rows in flight per CTA for that K
@@ -317,7 +320,84 @@ atom_status_t gemm_pairs(DeviceState *dev, bool pmode, int *pairs) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- W8A8 GEMM
+
+atom_status_t launch_w8a8(const int8_t *qa, const float *sa, const int8_t *qw, const float *sw,
+                          void *y, int64_t M, int64_t N, int64_t K, atom_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0) return ATOM_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return ATOM_OK;
+  // K: rows of 16-byte multiples for the TMA, and an int32 sum that cannot
+  // overflow (K * 127 * 127 < 2^31); N: 16-byte rows of fp16 Y.
+  if (K < 16 || K % 16 != 0 || K > 131072 || N % 8 != 0 || M > INT32_MAX || N > INT32_MAX)
+    return ATOM_ERR_SHAPE;
+  if (!qa || !sa || !qw || !sw || !y) return ATOM_ERR_INVALID_ARG;
+  if (!aligned(qa, 16) || !aligned(qw, 16) || !aligned(y, 16) || !aligned(sa, 4) ||
+      !aligned(sw, 16))
+    return ATOM_ERR_ALIGN;
+
+  DeviceState *dev = nullptr;
+  atom_status_t st = current_device(&dev);
+  if (st != ATOM_OK) return st;
+  using namespace atomk::w8a8_cfg;
+  int pairs = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!dev->w8a8_attr) {
+      const void *fn = reinterpret_cast<const void *>(atomk::w8a8_gemm_kernel);
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kSmemBytes)) != cudaSuccess)
+        return ATOM_ERR_CUDA;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * dev->sm_count, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 2;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg) != cudaSuccess || clusters < 1)
+        clusters = dev->sm_count / 2;
+      dev->w8a8_clusters = clusters;
+      dev->w8a8_attr = true;
+    }
+    pairs = dev->w8a8_clusters;
+  }
+
+  atomk::W8A8Maps maps;
+  const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  if (!encode_2d(&maps.a, u8, qa, K, M, K, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&maps.w, u8, qw, K, N, K, 128, BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&maps.y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, y, N, M, N * 2, 64, 32,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return ATOM_ERR_CUDA;
+  atomk::W8A8Params p;
+  p.sa = sa;
+  p.sw = sw;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.ksteps = static_cast<int>((K + 127) / 128);
+  p.m_tiles = static_cast<int>((M + kPairM - 1) / kPairM);
+  const int64_t tiles = static_cast<int64_t>(p.m_tiles) * ((N + BN - 1) / BN);
+  if (tiles > INT32_MAX) return ATOM_ERR_SHAPE;
+  p.tiles = static_cast<int>(tiles);
+  const int64_t used = tiles < pairs ? tiles : pairs;
+  atomk::w8a8_gemm_kernel<<<static_cast<int>(2 * used), kThreads, kSmemBytes,
+                            reinterpret_cast<cudaStream_t>(stream)>>>(maps, p);
+  return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
+}
+
 extern "C" {
+
+atom_status_t atom_w8a8_gemm(const int8_t *qa, const float *sa, const int8_t *qw,
+                             const float *sw, void *y, int64_t M, int64_t N, int64_t K,
+                             atom_stream_t stream) {
+  return launch_w8a8(qa, sa, qw, sw, y, M, N, K, stream);
+}
 
 atom_status_t atom_reorder_quant(const void *x, int64_t M, int64_t K, int64_t ld_x,
                                  const int32_t *outlier_idx, int32_t n_outlier, int32_t group,

@@ -130,3 +130,15 @@ def random_case(seed: int, M: int, N: int, K: int, dist: str = "t", param: float
     W = wt.astype(np.float16)
     assert np.isfinite(A).all() and np.isfinite(W).all()
     return A, W, idx.astype(np.int32)
+
+
+def int8_case(seed: int, M: int, N: int, K: int):
+    """Operands of the W8A8 comparator: int8 qa [M, K] and qw [N, K] uniform on
+    [-127, 127], and positive fp32 row scales sa [M] and column scales sw [N]
+    (log-uniform over two decades), all from Generator(PCG64(seed))."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    qa = rng.integers(-127, 128, size=(M, K), dtype=np.int16).astype(np.int8)
+    qw = rng.integers(-127, 128, size=(N, K), dtype=np.int16).astype(np.int8)
+    sa = (10.0 ** rng.uniform(-4.0, -2.0, size=M)).astype(np.float32)
+    sw = (10.0 ** rng.uniform(-4.0, -2.0, size=N)).astype(np.float32)
+    return qa, qw, sa, sw
