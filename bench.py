@@ -176,6 +176,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cublas", action="store_true",
                     help="skip the fp16 cuBLAS GEMM of the same shape reported beside the result")
+    ap.add_argument("--no-w8a8", action="store_true",
+                    help="skip the W8A8 comparator GEMM (and torch._int_mm) of the same shape")
     ap.add_argument("--m", type=int, default=None,
                     help="use only the first M activation rows (small profiling cases)")
     args = ap.parse_args()
@@ -327,6 +329,45 @@ def main():
                           "operands resident in HBM"}
         del W16, y16
 
+    # -------- W8A8 comparator of the same shape, and torch._int_mm (cuBLASLt int8)
+    w8a8 = None
+    if not args.no_w8a8:
+        qa8_h, qw8_h, sa8_h, sw8_h = inputs.int8_case(4000 + args.workload, w.M, w.N, w.K)
+        qa8 = torch.from_numpy(qa8_h).to(dev)
+        qw8 = torch.from_numpy(qw8_h).to(dev)
+        sa8 = torch.from_numpy(sa8_h).to(dev)
+        sw8 = torch.from_numpy(sw8_h).to(dev)
+        y8 = torch.empty((w.M, w.N), dtype=torch.float16, device=dev)
+        n_w8 = max(3, min(20, n_steps // 10))
+
+        def time_it(fn):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(n_w8):
+                fn()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            return a0.elapsed_time(a1) / n_w8
+
+        w8_ms = time_it(lambda: atom.atom_w8a8_gemm(qa8, sa8, qw8, sw8, y=y8, stream=stream))
+        mm_ms = time_it(lambda: torch._int_mm(qa8, qw8.t()))
+        ops8 = 2.0 * w.M * w.N * w.K
+        w8a8 = {"value": round(ops8 / (w8_ms * 1e-3) / 1e12, 2), "unit": "TOPS",
+                "ms": round(w8_ms, 4), "steps": n_w8,
+                "kind": "atom_w8a8_gemm: int8 x int8, per-row x per-column fp32 scales, fp16 out, "
+                        "same M, N, K, seeded uniform int8 operands resident in HBM",
+                "torch_int_mm": {"value": round(ops8 / (mm_ms * 1e-3) / 1e12, 2),
+                                 "unit": "TOPS", "ms": round(mm_ms, 4),
+                                 "kind": "torch._int_mm int8 x int8 -> int32 (cuBLASLt), "
+                                         "no scales"}}
+        del qa8, qw8, y8
+        if atom.atom_device_status(clear=True) != 0:
+            raise RuntimeError("device status set by the W8A8 comparator")
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -395,6 +436,9 @@ def main():
     if cublas is not None:
         cublas["w4a4_gemm_speedup"] = round(cublas["ms"] / gemm_avg, 3)
         line["fp16_cublas"] = cublas
+    if w8a8 is not None:
+        w8a8["frac_int8_peak"] = round(w8a8["value"] / int8_peak, 4)
+        line["w8a8"] = w8a8
     if world == 1 and not args.no_cpu_baseline:
         ops_s, rows, dt, cores = cpu_oracle_run(w, A_h, W_h, idx_h, args.cpu_budget)
         line["cpu_baseline"] = {"value": round(ops_s / 1e12, 6), "unit": "TOPS", "cores": cores,

@@ -417,9 +417,15 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     RingPos sr;
     for (int64_t it = 0; it < iters; ++it, w.next(p), sr.next(kNS)) {
       const int b = static_cast<int>(it & 1), sl = sr.idx;
-      const bool ok =
-          mbar_wait_inline(&tfull[b], static_cast<uint32_t>((it >> 1) & 1), abort_flag) &&
-          mbar_wait_inline(&sfull[sl], sr.phase, abort_flag);
+      const uint32_t tph = static_cast<uint32_t>((it >> 1) & 1);
+      // Both phases have usually completed by now: test them with two
+      // back-to-back try_waits and enter the (inline, timed) waits only if one
+      // has not; the inline wait alone costs ~160 cycles even on a completed
+      // phase, twice per group.
+      bool ok = mbar_try_wait(&tfull[b], tph) & mbar_try_wait(&sfull[sl], sr.phase);
+      if (!ok)
+        ok = mbar_wait_inline(&tfull[b], tph, abort_flag) &&
+             mbar_wait_inline(&sfull[sl], sr.phase, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) fail();
         break;
@@ -640,9 +646,12 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         const int s0 = p0.idx, s1 = p1.idx;
         TileWalk wn = w;
         wn.next(p);
-        bool ok = mbar_wait(&uempty[u], ur.phase ^ 1u, abort_flag) &&
-                  mbar_wait(&sempty[sl], sr.phase ^ 1u, abort_flag) &&
-                  mbar_wait(&pfull[s0], p0.phase, abort_flag);
+        bool ok = mbar_try_wait(&uempty[u], ur.phase ^ 1u) &
+                  mbar_try_wait(&sempty[sl], sr.phase ^ 1u) & mbar_try_wait(&pfull[s0], p0.phase);
+        if (!ok)
+          ok = mbar_wait(&uempty[u], ur.phase ^ 1u, abort_flag) &&
+               mbar_wait(&sempty[sl], sr.phase ^ 1u, abort_flag) &&
+               mbar_wait(&pfull[s0], p0.phase, abort_flag);
         if (ok && !int4_group) ok = mbar_wait(&pfull[s1], p1.phase, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) fail();
