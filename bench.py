@@ -202,7 +202,7 @@ def main():
 
     import torch
     import torch.distributed as dist
-    from w4a4_mixed_precision_b200 import atom
+    from w4a4_mixed_precision_b200 import atom, parallel
 
     if world > 1:
         import datetime
@@ -265,10 +265,7 @@ def main():
     elapsed_ms = t_start.elapsed_time(t_end)
     quant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n_steps)]
     gemm_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(n_steps)]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = parallel.max_over_ranks(elapsed_ms, dev)   # the slowest rank's time
 
     # -------- end-to-end through the public API with host buffers
     e2e = None
@@ -297,10 +294,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = parallel.max_over_ranks(e2e_ms, dev)
         e2e = {"value": round(2.0 * w.M * w.N * w.K * world / (e2e_ms * 1e-3) / 1e12, 2),
                "unit": "TOPS", "h2d_bytes_per_step": A_h.nbytes,
                "d2h_bytes_per_step": w.M * w.N * 2, "ms_per_step": round(e2e_ms, 4),
