@@ -219,6 +219,32 @@ ATOM_API atom_status_t atom_w8a8_gemm(const int8_t *qa, const float *sa, const i
                                       int64_t K, atom_stream_t stream);
 
 /*
+ * atom_kv_quant / atom_kv_dequant -- INT4 KV cache, one group per (token, head)
+ * vector of head_dim = 128 elements. The pages place Atom under KV-cache
+ * quantization ("Atom: Low-bit Quantization for Efficient and Accurate LLM
+ * Serving", key facts) without a KV recipe; the reading used is the Atom INT4
+ * group encoding ("Atom (mixed-precision block-outlier low-bit quantization
+ * for serving)", Bits and Weight group size) with no reorder and no outliers:
+ *
+ *   scale[g] = fl32(amax / 7), inv = fl32(7 / amax)   (0, 0 for an all-zero group)
+ *   q = rint(fl32(x * inv)) in [-7, 7], ties to even
+ *   q4[g][i] = (q[2i] & 0xF) | (q[2i+1] << 4)
+ *   atom_kv_dequant: out[g][j] = fp16_rn(fl32(q[j] * scale[g]))
+ *
+ *   x, out   fp16 [groups][128] device (a cache [tokens][heads][128] flattened).
+ *   q4       uint8 [groups][64] device.
+ *   scales   fp32 [groups] device.
+ * groups = 0 is a no-op; negative groups or a null pointer ->
+ * ATOM_ERR_INVALID_ARG; x and out must be 16-byte aligned, q4 8-byte, scales
+ * 4-byte (else ATOM_ERR_ALIGN). Inputs must be finite. Stream-ordered,
+ * allocates nothing.
+ */
+ATOM_API atom_status_t atom_kv_quant(const void *x, int64_t groups, uint8_t *q4, float *scales,
+                                     atom_stream_t stream);
+ATOM_API atom_status_t atom_kv_dequant(const uint8_t *q4, const float *scales, int64_t groups,
+                                       void *out, atom_stream_t stream);
+
+/*
  * atom_device_status -- first device-detected error since the last clear on the
  * current device (ATOM_OK if none). Synchronises the current device. With
  * clear != 0 the status is reset to ATOM_OK afterwards.

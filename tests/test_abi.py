@@ -137,3 +137,15 @@ def test_w8a8_checks_arguments_on_the_host(lib):
     assert w8a8(lib, qw=A16 + 8) == ALIGN
     assert w8a8(lib, sw=A16 + 4) == ALIGN   # sw is read as 16-byte vectors
     assert w8a8(lib, sa=MIS) == ALIGN
+
+
+def test_kv_checks_arguments_on_the_host(lib):
+    assert lib.atom_kv_quant(A16, 0, A16, A16, None) == OK
+    assert lib.atom_kv_dequant(A16, A16, 0, A16, None) == OK
+    assert lib.atom_kv_quant(A16, -1, A16, A16, None) == INVALID
+    assert lib.atom_kv_quant(0, 4, A16, A16, None) == INVALID
+    assert lib.atom_kv_dequant(A16, 0, 4, A16, None) == INVALID
+    assert lib.atom_kv_quant(A16 + 8, 4, A16, A16, None) == ALIGN     # x: 16 bytes
+    assert lib.atom_kv_quant(A16, 4, A16 + 4, A16, None) == ALIGN     # q4: 8 bytes
+    assert lib.atom_kv_quant(A16, 4, A16, MIS, None) == ALIGN         # scales: 4 bytes
+    assert lib.atom_kv_dequant(A16, A16, 4, A16 + 8, None) == ALIGN   # out: 16 bytes

@@ -53,6 +53,9 @@ SIGNATURES = {
                                                     ct.c_int32, ct.c_void_p], ct.c_int),
     "atom_w8a8_gemm": ([ct.c_void_p] * 5 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_void_p],
                        ct.c_int),
+    "atom_kv_quant": ([ct.c_void_p, ct.c_int64, ct.c_void_p, ct.c_void_p, ct.c_void_p], ct.c_int),
+    "atom_kv_dequant": ([ct.c_void_p, ct.c_void_p, ct.c_int64, ct.c_void_p, ct.c_void_p],
+                        ct.c_int),
     "atom_device_status": ([ct.c_int], ct.c_int),
     "atom_status_string": ([ct.c_int], ct.c_char_p),
     "atom_version": ([], ct.c_int),
@@ -236,6 +239,38 @@ def atom_w8a8_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: tor
         _dev(sw, torch.float32, "sw"), _dev(y, torch.float16, "y"), M, N, K, _stream(stream))
     _check("atom_w8a8_gemm", st)
     return y
+
+
+def atom_kv_quant(x: torch.Tensor, q4: Optional[torch.Tensor] = None,
+                  scales: Optional[torch.Tensor] = None, stream=None):
+    """INT4 KV-cache quantization of fp16 [..., 128] (one group per 128-vector):
+    returns (q4 uint8 [..., 64], scales fp32 [...]) (see include/atom.h)."""
+    if x.shape[-1] != 128:
+        raise ValueError("atom_kv_quant: the last axis must be head_dim = 128")
+    lead = tuple(x.shape[:-1])
+    groups = x.numel() // 128
+    if q4 is None:
+        q4 = torch.empty(lead + (64,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(lead, dtype=torch.float32, device=x.device)
+    st = lib().atom_kv_quant(_dev(x, torch.float16, "x"), groups, _dev(q4, torch.uint8, "q4"),
+                             _dev(scales, torch.float32, "scales"), _stream(stream))
+    _check("atom_kv_quant", st)
+    return q4, scales
+
+
+def atom_kv_dequant(q4: torch.Tensor, scales: torch.Tensor, out: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """fp16 [..., 128] from atom_kv_quant's codes and scales."""
+    if q4.shape[-1] != 64 or tuple(scales.shape) != tuple(q4.shape[:-1]):
+        raise ValueError("atom_kv_dequant: q4 [..., 64] and scales [...] must match")
+    groups = scales.numel()
+    if out is None:
+        out = torch.empty(tuple(q4.shape[:-1]) + (128,), dtype=torch.float16, device=q4.device)
+    st = lib().atom_kv_dequant(_dev(q4, torch.uint8, "q4"), _dev(scales, torch.float32, "scales"),
+                               groups, _dev(out, torch.float16, "out"), _stream(stream))
+    _check("atom_kv_dequant", st)
+    return out
 
 
 def atom_gemm_workspace_bytes(M: int, N: int, K: int) -> int:

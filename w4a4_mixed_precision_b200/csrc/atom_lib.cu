@@ -9,6 +9,7 @@
 #include "gemm.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
+#include "kv.cuh"
 #include "w8a8.cuh"
 
 namespace {
@@ -391,7 +392,45 @@ atom_status_t launch_w8a8(const int8_t *qa, const float *sa, const int8_t *qw, c
   return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- INT4 KV cache
+
+int kv_grid(const DeviceState *dev, int64_t groups) {
+  const int64_t want = (groups * 8 + atomk::kKvThreads - 1) / atomk::kKvThreads;
+  const int64_t cap = static_cast<int64_t>(dev->sm_count) * 8;
+  return static_cast<int>(want < cap ? want : cap);
+}
+
 extern "C" {
+
+atom_status_t atom_kv_quant(const void *x, int64_t groups, uint8_t *q4, float *scales,
+                            atom_stream_t stream) {
+  if (groups < 0) return ATOM_ERR_INVALID_ARG;
+  if (groups == 0) return ATOM_OK;
+  if (!x || !q4 || !scales) return ATOM_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(q4, 8) || !aligned(scales, 4)) return ATOM_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  atom_status_t st = current_device(&dev);
+  if (st != ATOM_OK) return st;
+  atomk::kv_quant_kernel<<<kv_grid(dev, groups), atomk::kKvThreads, 0,
+                           reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __half *>(x), groups, q4, scales);
+  return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
+}
+
+atom_status_t atom_kv_dequant(const uint8_t *q4, const float *scales, int64_t groups, void *out,
+                              atom_stream_t stream) {
+  if (groups < 0) return ATOM_ERR_INVALID_ARG;
+  if (groups == 0) return ATOM_OK;
+  if (!q4 || !scales || !out) return ATOM_ERR_INVALID_ARG;
+  if (!aligned(q4, 8) || !aligned(scales, 4) || !aligned(out, 16)) return ATOM_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  atom_status_t st = current_device(&dev);
+  if (st != ATOM_OK) return st;
+  atomk::kv_dequant_kernel<<<kv_grid(dev, groups), atomk::kKvThreads, 0,
+                             reinterpret_cast<cudaStream_t>(stream)>>>(
+      q4, scales, groups, static_cast<__half *>(out));
+  return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
+}
 
 atom_status_t atom_w8a8_gemm(const int8_t *qa, const float *sa, const int8_t *qw,
                              const float *sw, void *y, int64_t M, int64_t N, int64_t K,

@@ -142,3 +142,18 @@ def int8_case(seed: int, M: int, N: int, K: int):
     sa = (10.0 ** rng.uniform(-4.0, -2.0, size=M)).astype(np.float32)
     sw = (10.0 ** rng.uniform(-4.0, -2.0, size=N)).astype(np.float32)
     return qa, qw, sa, sw
+
+
+def kv_cache(seed: int, tokens: int, heads: int, head_dim: int = 128) -> np.ndarray:
+    """fp16 [tokens, heads, head_dim] key/value vectors: standard normal draws,
+    each (token, head) vector scaled by a log-uniform factor over four decades,
+    and one seeded element per vector in 64 multiplied by 8 (an outlier);
+    Generator(PCG64(seed))."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    v = rng.standard_normal((tokens, heads, head_dim))
+    v *= 10.0 ** rng.uniform(-2.0, 2.0, size=(tokens, heads, 1))
+    spikes = rng.random((tokens, heads, head_dim)) < 1.0 / 64
+    v[spikes] *= 8.0
+    out = v.astype(np.float16)
+    assert np.isfinite(out).all()
+    return out
