@@ -178,6 +178,8 @@ def main():
                     help="skip the fp16 cuBLAS GEMM of the same shape reported beside the result")
     ap.add_argument("--no-w8a8", action="store_true",
                     help="skip the W8A8 comparator GEMM (and torch._int_mm) of the same shape")
+    ap.add_argument("--no-kv", action="store_true",
+                    help="skip the INT4 KV-cache quantize/dequantize measurement")
     ap.add_argument("--m", type=int, default=None,
                     help="use only the first M activation rows (small profiling cases)")
     args = ap.parse_args()
@@ -362,6 +364,46 @@ def main():
         if atom.atom_device_status(clear=True) != 0:
             raise RuntimeError("device status set by the W8A8 comparator")
 
+    # -------- INT4 KV cache: 131072 tokens x 8 KV heads x head_dim 128 (268 MB fp16)
+    kv = None
+    if not args.no_kv:
+        kv_tokens, kv_heads = 131072, 8
+        kv_x = [torch.from_numpy(inputs.kv_cache(5000 + i, kv_tokens, kv_heads).view(np.uint16))
+                .to(dev).view(torch.float16) for i in range(2)]
+        kv_q = [atom.atom_kv_quant(x, stream=stream) for x in kv_x]
+        kv_y = [torch.empty_like(x) for x in kv_x]
+        n_kv = max(3, min(20, n_steps // 10))
+
+        def time_kv(fn):
+            for i in range(3):
+                fn(i)
+            torch.cuda.synchronize()
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for i in range(n_kv):
+                fn(i)
+            a1.record(stream)
+            torch.cuda.synchronize()
+            return a0.elapsed_time(a1) / n_kv
+
+        q_ms = time_kv(lambda i: atom.atom_kv_quant(kv_x[i % 2], q4=kv_q[i % 2][0],
+                                                     scales=kv_q[i % 2][1], stream=stream))
+        d_ms = time_kv(lambda i: atom.atom_kv_dequant(kv_q[i % 2][0], kv_q[i % 2][1],
+                                                       out=kv_y[i % 2], stream=stream))
+        kv_groups = kv_tokens * kv_heads
+        kv_bytes = kv_groups * (256 + 64 + 4)   # fp16 vectors + packed codes + scales
+        kv = {"shape": f"{kv_tokens} tokens x {kv_heads} heads x 128", "groups": kv_groups,
+              "bytes_per_call": kv_bytes,
+              "quant": {"value": round(kv_bytes / (q_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                        "ms": round(q_ms, 4)},
+              "dequant": {"value": round(kv_bytes / (d_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                          "ms": round(d_ms, 4)},
+              "l2": "two caches of 268 MB alternate, larger than L2"}
+        del kv_x, kv_q, kv_y
+        if atom.atom_device_status(clear=True) != 0:
+            raise RuntimeError("device status set by the KV-cache kernels")
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -433,6 +475,10 @@ def main():
     if w8a8 is not None:
         w8a8["frac_int8_peak"] = round(w8a8["value"] / int8_peak, 4)
         line["w8a8"] = w8a8
+    if kv is not None:
+        kv["quant"]["frac_hbm"] = round(kv["quant"]["value"] / peaks["hbm_gbs"], 4)
+        kv["dequant"]["frac_hbm"] = round(kv["dequant"]["value"] / peaks["hbm_gbs"], 4)
+        line["kv_int4"] = kv
     if world == 1 and not args.no_cpu_baseline:
         ops_s, rows, dt, cores = cpu_oracle_run(w, A_h, W_h, idx_h, args.cpu_budget)
         line["cpu_baseline"] = {"value": round(ops_s / 1e12, 6), "unit": "TOPS", "cores": cores,
