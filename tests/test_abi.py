@@ -149,3 +149,16 @@ def test_kv_checks_arguments_on_the_host(lib):
     assert lib.atom_kv_quant(A16, 4, A16 + 4, A16, None) == ALIGN     # q4: 8 bytes
     assert lib.atom_kv_quant(A16, 4, A16, MIS, None) == ALIGN         # scales: 4 bytes
     assert lib.atom_kv_dequant(A16, A16, 4, A16 + 8, None) == ALIGN   # out: 16 bytes
+
+
+def test_header_compiles_as_plain_c(tmp_path):
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_atom.c"
+    src.write_text('#include "atom.h"\nint main(void) { return atom_status_string(ATOM_OK) == 0; }\n')
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-I",
+                        os.path.join(ROOT, "include"), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
