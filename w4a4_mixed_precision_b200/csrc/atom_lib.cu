@@ -7,6 +7,7 @@
 
 #include "atom.h"
 #include "gemm.cuh"
+#include "gemm_small.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 #include "kv.cuh"
@@ -24,6 +25,7 @@ struct DeviceState {
   int smem_optin = 0;
   bool gemm_attr[2] = {false, false};
   int gemm_clusters[2] = {0, 0};  // co-resident CTA pairs of the GEMM kernel
+  bool small_attr = false;       // shared-memory limit set for the small-M GEMM kernels
   bool w8a8_attr = false;
   int w8a8_clusters = 0;          // co-resident CTA pairs of the W8A8 kernel
   uint32_t quant_smem_set = 0;
@@ -189,6 +191,85 @@ int gemm_splits(int64_t M, int64_t N, int64_t K, int pairs) {
 
 atom_status_t gemm_pairs(DeviceState *dev, bool pmode, int *pairs);
 
+// K splits of the small-M GEMM (gemm_small.cuh): one 128-row weight tile per
+// CTA, as many K ranges (of at least 2 groups, at most kMaxSplits) as keep
+// every SM busy without a second wave. 1 = no split.
+int small_splits(int64_t N, int64_t K, int sms) {
+  const int64_t n_tiles = (N + atomk::small_cfg::BW - 1) / atomk::small_cfg::BW;
+  if (n_tiles <= 0 || n_tiles >= sms) return 1;
+  int64_t s = sms / n_tiles;
+  const int64_t by_k = (K / 128) / 2;
+  if (s > by_k) s = by_k;
+  if (s > kMaxSplits) s = kMaxSplits;
+  return s < 2 ? 1 : static_cast<int>(s);
+}
+
+// The GEMM for M <= 64 tokens: weights on the MMA's M side (see gemm_small.cuh).
+atom_status_t launch_gemm_small(DeviceState *dev, const uint8_t *qa4, const int8_t *qa8,
+                                const float *sa, const uint8_t *qw4, const int8_t *qw8,
+                                const float *sw, void *y, int64_t M, int64_t N, int64_t K,
+                                void *workspace, size_t workspace_bytes, atom_stream_t stream) {
+  using namespace atomk::small_cfg;
+  const int64_t q4_row = (K - 128) / 2;
+  int splits = small_splits(N, K, dev->sm_count);
+  if (splits > 1 && (workspace == nullptr ||
+                     workspace_bytes < static_cast<size_t>(splits) * M * N * sizeof(float) ||
+                     !aligned(workspace, 16)))
+    splits = 1;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!dev->small_attr) {
+      const void *fns[3] = {reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<16>),
+                            reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<32>),
+                            reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<64>)};
+      for (const void *fn : fns)
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kSmemBytes)) != cudaSuccess)
+          return ATOM_ERR_CUDA;
+      dev->small_attr = true;
+    }
+  }
+  atomk::SmallMaps maps;
+  const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  if (!encode_2d(&maps.w4, u8, qw4, q4_row, N, q4_row, 64, BW, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_2d(&maps.a4, u8, qa4, q4_row, M, q4_row, 64, kMaxTokens,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_2d(&maps.w8, u8, qw8, 128, N, 128, 128, BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&maps.a8, u8, qa8, 128, M, 128, 128, kMaxTokens, CU_TENSOR_MAP_SWIZZLE_128B))
+    return ATOM_ERR_CUDA;
+  atomk::SmallParams p;
+  p.sa = sa;
+  p.sw = sw;
+  p.y = static_cast<__half *>(y);
+  p.ws = splits > 1 ? static_cast<float *>(workspace) : nullptr;
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.G = static_cast<int>(K / 128);
+  p.n_tiles = static_cast<int>((N + BW - 1) / BW);
+  p.splits = splits;
+  p.items = p.n_tiles * splits;
+  const int grid = p.items < dev->sm_count ? p.items : dev->sm_count;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (M <= 16)
+    atomk::w4a4_gemm_small_kernel<16><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
+  else if (M <= 32)
+    atomk::w4a4_gemm_small_kernel<32><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
+  else
+    atomk::w4a4_gemm_small_kernel<64><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
+  if (cudaGetLastError() != cudaSuccess) return ATOM_ERR_CUDA;
+  if (splits > 1) {
+    const int64_t count8 = M * N / 8;
+    int64_t blocks = (count8 + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(dev->sm_count) * 8;
+    if (blocks > cap) blocks = cap;
+    atomk::splitk_reduce_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
+        p.ws, static_cast<__half *>(y), count8, M * N, splits);
+    if (cudaGetLastError() != cudaSuccess) return ATOM_ERR_CUDA;
+  }
+  return ATOM_OK;
+}
+
 atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa,
                           const uint8_t *qw4, const int8_t *qw8, const float *sw, void *y,
                           int32_t *partials, int64_t M, int64_t N, int64_t K, int32_t n_outlier,
@@ -214,6 +295,9 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
 
   using namespace atomk::gemm_cfg;
   const bool pmode = partials != nullptr;
+  if (!pmode && M <= atomk::small_cfg::kMaxTokens)
+    return launch_gemm_small(dev, qa4, qa8, sa, qw4, qw8, sw, y, M, N, K, workspace,
+                             workspace_bytes, stream);
   int pairs = 0;
   if ((st = gemm_pairs(dev, pmode, &pairs)) != ATOM_OK) return st;
 
@@ -472,8 +556,14 @@ size_t atom_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K < 256) return 0;
   DeviceState *dev = nullptr;
   int pairs = 0;
-  if (current_device(&dev) != ATOM_OK || gemm_pairs(dev, false, &pairs) != ATOM_OK) return 0;
-  const int splits = gemm_splits(M, N, K, pairs);
+  if (current_device(&dev) != ATOM_OK) return 0;
+  int splits = 1;
+  if (M <= atomk::small_cfg::kMaxTokens) {
+    splits = small_splits(N, K, dev->sm_count);
+  } else {
+    if (gemm_pairs(dev, false, &pairs) != ATOM_OK) return 0;
+    splits = gemm_splits(M, N, K, pairs);
+  }
   return splits > 1 ? static_cast<size_t>(splits) * M * N * sizeof(float) : 0;
 }
 

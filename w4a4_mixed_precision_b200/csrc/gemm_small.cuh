@@ -1,0 +1,452 @@
+// gemm_small.cuh -- the W4A4 GEMM for a few tokens (M <= 64, decode).
+//
+// Same arithmetic as w4a4_gemm_kernel (gemm.cuh): exact int32 per-group
+// partials P_g on the tensor cores and Y = sum_g sa * sw * P_g in fp32, with
+// every element computed by the same fp32 operations in the same group order
+// (so an unsplit call gives bit-identical Y). What changes is the shape of the
+// work. A 256x256 tile would leave at most 64 of its rows valid and drain 256
+// columns per group; here the weights are the MMA's M side and the tokens its
+// N side:
+//
+//   one CTA owns 128 weight rows (output columns n0..n0+127) and one range of
+//   K groups; per group, four tcgen05.mma.cta_group::1.kind::i8 with M = 128
+//   (weight rows), N = NT (the tokens rounded up to 16, 32 or 64), K = 32
+//   accumulate into an NT-column TMEM accumulator (two alternate); four drain
+//   warps, one per TMEM lane quarter, hold one weight row each and NT token
+//   columns of fp32 accumulators; K is split so that about one CTA per SM
+//   works, each range's fp32 partial tile going to the caller's workspace for
+//   the ordered reduction kernel of gemm.cuh.
+//
+// Roles (12 warps): warp 0 lane 0 TMA producer; warp 1 lane 0 MMA issuer;
+// warps 2..7 unpack (nibbles to 16*q bytes, K-major, 128-byte swizzle, as in
+// gemm.cuh; the INT8 outlier group is copied) and lay the scales out; warps
+// 8..11 drain. Accumulators start at the conversion bias as in gemm.cuh.
+#pragma once
+
+#include "gemm.cuh"
+
+namespace atomk {
+
+namespace small_cfg {
+constexpr int BW = 128;                 // weight rows (output columns) per CTA
+constexpr int kMaxTokens = 64;          // token rows per call
+constexpr int kThreads = 384;
+constexpr int kUnpackThreads = 192;     // warps 2..7
+constexpr int kUnpackWarps = kUnpackThreads / 32;
+constexpr int kDrainWarps = 4;          // warps 8..11
+constexpr int kNP = 4, kNU = 3, kNS = 6;
+// packed slot: INT4 W (128 x 64 B) at 0 and INT4 A (64 x 64 B) at kPackAOff;
+// the INT8 group takes two slots: W8 (128 x 128 B), then A8 (64 x 128 B)
+constexpr uint32_t kPackAOff = BW * 64;
+constexpr uint32_t kPSlot = 17 * 1024;
+// operand slot: int8 W (128 x 128 B) then int8 A (64 x 128 B), K-major, 128-byte swizzle
+constexpr uint32_t kOpAOff = BW * 128;
+constexpr uint32_t kUSlot = kOpAOff + kMaxTokens * 128;
+// scale slot: per token pair (sa'[2j], sa'[2j+1], nc[2j], nc[2j+1]), then sw by weight row
+constexpr uint32_t kSwOff = kMaxTokens * 8;
+constexpr uint32_t kSSlot = kSwOff + BW * 4;
+constexpr uint32_t kBarBytes = 1024;
+constexpr uint32_t kPOff = kBarBytes;
+constexpr uint32_t kUOff = kPOff + kNP * kPSlot;
+constexpr uint32_t kSOff = kUOff + kNU * kUSlot;
+constexpr uint32_t kSmemBytes = kSOff + kNS * kSSlot + 1024;   // + alignment slack
+constexpr uint32_t kTmemCols = 2 * kMaxTokens;
+constexpr int kPackedChunks = (BW + kMaxTokens) * 4;            // 16-byte chunks, INT4 group
+constexpr int kInt8Chunks = (BW + kMaxTokens) * 8;              // 16-byte chunks, INT8 group
+static_assert(kPSlot % 1024 == 0 && kUSlot % 1024 == 0 && kOpAOff % 1024 == 0, "1024-byte slots");
+static_assert(kPackAOff + kMaxTokens * 64 <= kPSlot && BW * 128 <= kPSlot, "packed slot");
+static_assert(kPackedChunks % kUnpackThreads == 0 && kInt8Chunks % kUnpackThreads == 0, "chunks");
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+}  // namespace small_cfg
+
+struct SmallMaps {
+  CUtensorMap w4;   // packed INT4 W: uint8 [N][(K-128)/2], boxes of 128 rows x 64 bytes
+  CUtensorMap a4;   // packed INT4 A: uint8 [M][(K-128)/2], boxes of 64 rows x 64 bytes
+  CUtensorMap w8;   // INT8 W: [N][128], boxes 128 x 128 bytes, 128-byte swizzle
+  CUtensorMap a8;   // INT8 A: [M][128], boxes 64 x 128 bytes, 128-byte swizzle
+};
+
+struct SmallParams {
+  const float *sa;   // [G][M]
+  const float *sw;   // [G][N]
+  __half *y;         // splits == 1
+  float *ws;         // splits > 1: fp32 partial outputs [splits][M][N]
+  int M, N, K, G;
+  int n_tiles, splits, items;
+};
+
+// The (item, group) sequence of one CTA; every role walks the same one. Item i
+// is weight tile i / splits and K range i % splits.
+struct SmallWalk {
+  int item, g, g_end, split, n0;
+  __device__ __forceinline__ void set(const SmallParams &p) {
+    const int tile = item / p.splits;
+    split = item - tile * p.splits;
+    n0 = tile * small_cfg::BW;
+    g = split * p.G / p.splits;
+    g_end = (split + 1) * p.G / p.splits;
+  }
+  __device__ __forceinline__ void start(const SmallParams &p) {
+    item = blockIdx.x;
+    set(p);
+  }
+  __device__ __forceinline__ bool last() const { return g == g_end - 1; }
+  __device__ __forceinline__ void next(const SmallParams &p) {
+    if (++g == g_end) {
+      item += gridDim.x;
+      set(p);
+    }
+  }
+};
+
+__device__ __forceinline__ int64_t small_iterations(const SmallParams &p) {
+  int64_t n = 0;
+  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+    const int s = it % p.splits;
+    n += (s + 1) * p.G / p.splits - s * p.G / p.splits;
+  }
+  return n;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(small_cfg::kThreads, 1)
+w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams p) {
+  using namespace small_cfg;
+  static_assert(NT == 16 || NT == 32 || NT == 64, "token tile");
+  constexpr uint32_t kIdescSmall = idesc_i8(BW, NT);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+
+  uint64_t *pfull = reinterpret_cast<uint64_t *>(smem);   // [kNP] TMA -> unpackers
+  uint64_t *pempty = pfull + kNP;                         // [kNP] unpackers -> producer
+  uint64_t *ufull = pempty + kNP;                         // [kNU] operands ready -> MMA
+  uint64_t *uempty = ufull + kNU;                         // [kNU] MMA commit -> unpackers
+  uint64_t *sfull = uempty + kNU;                         // [kNS] scales ready -> drain
+  uint64_t *sempty = sfull + kNS;                         // [kNS] drain -> unpackers
+  uint64_t *tfull = sempty + kNS;                         // [2] accumulator complete
+  uint64_t *tempty = tfull + 2;                           // [2] accumulator drained
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  uint8_t *pring = smem + kPOff;
+  uint8_t *uring = smem + kUOff;
+  uint8_t *sring = smem + kSOff;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNP; ++s) {
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pempty[s], kUnpackWarps);
+    }
+    for (int s = 0; s < kNU; ++s) {
+      mbar_init(&ufull[s], kUnpackWarps);
+      mbar_init(&uempty[s], 1);
+    }
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&sfull[s], kUnpackWarps);
+      mbar_init(&sempty[s], kDrainWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], kDrainWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tbase = *tmem_slot;
+  const int64_t iters = small_iterations(p);
+
+  // both accumulators start at the conversion bias (see gemm.cuh)
+  if (warp >= 8) {
+    const uint32_t lanes = tbase + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+#pragma unroll
+    for (int b = 0; b < 2; ++b)
+#pragma unroll
+      for (int c = 0; c < NT / 4; ++c) tmem_st_x4_fill(lanes + b * kMaxTokens + 4 * c, gemm_cfg::kBias);
+    tmem_st_wait();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+
+  auto fail = [&](void) {
+    report_status(6 /* ATOM_ERR_TIMEOUT */);
+    *abort_flag = 1;
+  };
+
+  if (warp >= 8) {
+    // ================================================================ drain
+    // Warp 8 + q owns TMEM lanes [32q, 32q+32): thread `lane` holds weight row
+    // n0 + 32q + lane and the NT token columns of its accumulator.
+    const int q = warp - 8;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
+    const int lrow = 32 * q + lane;
+    float2 acc[NT / 2];
+#pragma unroll
+    for (int i = 0; i < NT / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+    SmallWalk w;
+    w.start(p);
+    RingPos sr;
+    for (int64_t it = 0; it < iters; ++it, w.next(p), sr.next(kNS)) {
+      const int b = static_cast<int>(it & 1), sl = sr.idx;
+      const uint32_t tph = static_cast<uint32_t>((it >> 1) & 1);
+      bool ok = mbar_try_wait(&tfull[b], tph) & mbar_try_wait(&sfull[sl], sr.phase);
+      if (!ok)
+        ok = mbar_wait(&tfull[b], tph, abort_flag) && mbar_wait(&sfull[sl], sr.phase, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) fail();
+        break;
+      }
+      tc_fence_after_sync();
+      const uint8_t *ss = sring + sl * kSSlot;
+      // per token pair: (sa'[2j], sa'[2j+1], -C*sa'[2j], -C*sa'[2j+1]); sa' as in gemm.cuh
+      const float4 *sap = reinterpret_cast<const float4 *>(ss);
+      const float swr = reinterpret_cast<const float *>(ss + kSwOff)[lrow];
+      const float2 sw2 = make_float2(swr, swr);
+      const uint32_t tcol = tbase + lane_base + b * kMaxTokens;
+      uint32_t ra[16], rb[16];
+      tmem_ld_x16(tcol, ra);
+      tmem_ld_wait(ra);
+#pragma unroll
+      for (int c = 0; c < NT / 16; ++c) {
+        uint32_t(&r)[16] = (c & 1) ? rb : ra;
+        uint32_t(&rn)[16] = (c & 1) ? ra : rb;
+        if (c + 1 < NT / 16) tmem_ld_x16(tcol + 16 * (c + 1), rn);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {   // token pair 8c + j: columns 16c + 2j, 16c + 2j + 1
+          const float4 s4 = sap[8 * c + j];
+          const float2 f = make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+          float2 &a = acc[8 * c + j];
+          a = f2_fma(f2_fma(f, make_float2(s4.x, s4.y), make_float2(s4.z, s4.w)), sw2, a);
+        }
+        if (c + 1 < NT / 16) tmem_ld_wait(rn);
+      }
+#pragma unroll
+      for (int e = 0; e < NT / 4; ++e) tmem_st_x4_fill(tcol + 4 * e, gemm_cfg::kBias);
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&tempty[b]);
+        mbar_arrive(&sempty[sl]);
+      }
+      if (w.last()) {
+        // this K range of the item is complete: write the thread's row of Y
+        // (tokens m < M), or the split's fp32 partial tile; consecutive lanes
+        // write consecutive columns
+        const int n = w.n0 + lrow;
+        const bool row_ok = n < p.N;
+#pragma unroll
+        for (int j = 0; j < NT / 2; ++j) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int m = 2 * j + h;
+            const float v = h ? acc[j].y : acc[j].x;
+            if (row_ok && m < p.M) {
+              if (p.splits == 1)
+                p.y[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(v);
+              else
+                p.ws[(static_cast<int64_t>(w.split) * p.M + m) * p.N + n] = v;
+            }
+          }
+          acc[j] = make_float2(0.f, 0.f);
+        }
+      }
+    }
+  } else if (warp == 0) {
+    // ================================================================ producer
+    if (lane == 0) {
+      SmallWalk wp;
+      wp.start(p);
+      RingPos pr;
+      int64_t ls = 0;
+      bool ok = true;
+      for (int64_t it = 0; ok && it < iters; ++it, wp.next(p)) {
+        const bool int4_group = wp.g < p.G - 1;
+        for (int part = 0; part < (int4_group ? 1 : 2); ++part) {
+          const int s = pr.idx;
+          if (!mbar_wait(&pempty[s], pr.phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t *slot = pring + s * kPSlot;
+          if (int4_group) {
+            mbar_arrive_expect_tx(&pfull[s], BW * 64u + kMaxTokens * 64u);
+            tma_load_2d(slot, &maps.w4, wp.g * 64, wp.n0, &pfull[s]);
+            tma_load_2d(slot + kPackAOff, &maps.a4, wp.g * 64, 0, &pfull[s]);
+          } else if (part == 0) {
+            mbar_arrive_expect_tx(&pfull[s], BW * 128u);
+            tma_load_2d(slot, &maps.w8, 0, wp.n0, &pfull[s]);
+          } else {
+            mbar_arrive_expect_tx(&pfull[s], kMaxTokens * 128u);
+            tma_load_2d(slot, &maps.a8, 0, 0, &pfull[s]);
+          }
+          ++ls;
+          pr.next(kNP);
+        }
+      }
+      if (!ok) {
+        fail();
+        for (int64_t j = (ls > kNP ? ls - kNP : 0); j < ls; ++j)
+          (void)mbar_wait(&pfull[j % kNP], static_cast<uint32_t>((j / kNP) & 1), nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      int64_t last_mma = -1;
+      bool ok = true;
+      RingPos ur;
+      for (int64_t it = 0; ok && it < iters; ++it, ur.next(kNU)) {
+        const int u = ur.idx, b = static_cast<int>(it & 1);
+        const uint32_t eph = static_cast<uint32_t>(((it >> 1) & 1) ^ 1);
+        if (!(mbar_try_wait(&ufull[u], ur.phase) & mbar_try_wait(&tempty[b], eph)) &&
+            (!mbar_wait(&ufull[u], ur.phase, abort_flag) ||
+             !mbar_wait(&tempty[b], eph, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t op = smem_addr(uring + u * kUSlot);
+        const uint64_t adesc = smem_desc_k_sw128(op);             // weights, 128 rows
+        const uint64_t bdesc = smem_desc_k_sw128(op + kOpAOff);   // tokens, NT rows
+        const uint32_t d = tbase + b * kMaxTokens;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mma_i8(d, adesc + 2 * k, bdesc + 2 * k, kIdescSmall, 1u);
+        tc_commit(&tfull[b]);
+        tc_commit(&uempty[u]);
+        last_mma = it;
+      }
+      if (!ok) fail();
+      // nothing may still write TMEM when it is released
+      if (last_mma >= 0)
+        (void)mbar_wait(&tfull[last_mma & 1], static_cast<uint32_t>((last_mma >> 1) & 1), nullptr);
+    }
+  } else {
+    // ================================================================ unpackers
+    const int lt = threadIdx.x - 64;
+    // This thread's raw scales of a group: sw of weight row n0 + lt (lt < 128),
+    // or sa of tokens 2j, 2j+1 (j = lt - 128 < 32). They are fetched one group
+    // ahead, so that their global-memory latency is not on the group's path.
+    auto load_scales = [&](const SmallWalk &g, float (&v)[2]) {
+      v[0] = v[1] = 0.f;
+      if (lt < BW) {
+        const int n = g.n0 + lt;
+        if (n < p.N) v[0] = __ldg(p.sw + static_cast<int64_t>(g.g) * p.N + n);
+      } else if (lt < BW + kMaxTokens / 2) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int m = 2 * (lt - BW) + h;
+          if (m < p.M) v[h] = __ldg(p.sa + static_cast<int64_t>(g.g) * p.M + m);
+        }
+      }
+    };
+    SmallWalk w;
+    w.start(p);
+    float sc[2];
+    if (iters > 0) load_scales(w, sc);
+    RingPos ur, sr, pr;
+    for (int64_t it = 0; it < iters; ++it, ur.next(kNU), sr.next(kNS), w.next(p)) {
+      float sc_next[2] = {0.f, 0.f};
+      if (it + 1 < iters) {
+        SmallWalk w1 = w;
+        w1.next(p);
+        load_scales(w1, sc_next);
+      }
+      const int u = ur.idx, sl = sr.idx;
+      const bool int4_group = w.g < p.G - 1;
+      const RingPos p0 = pr;
+      RingPos p1 = pr;
+      p1.next(kNP);
+      bool ok = mbar_try_wait(&uempty[u], ur.phase ^ 1u) &
+                mbar_try_wait(&sempty[sl], sr.phase ^ 1u) & mbar_try_wait(&pfull[p0.idx], p0.phase);
+      if (!ok)
+        ok = mbar_wait(&uempty[u], ur.phase ^ 1u, abort_flag) &&
+             mbar_wait(&sempty[sl], sr.phase ^ 1u, abort_flag) &&
+             mbar_wait(&pfull[p0.idx], p0.phase, abort_flag);
+      if (ok && !int4_group) ok = mbar_wait(&pfull[p1.idx], p1.phase, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) fail();
+        break;
+      }
+      const uint8_t *pk = pring + p0.idx * kPSlot;
+      uint8_t *op = uring + u * kUSlot;
+      if (int4_group) {
+        // nibbles -> bytes holding 16*q, K-major with the 128-byte swizzle
+#pragma unroll
+        for (int i = 0; i < kPackedChunks / kUnpackThreads; ++i) {
+          const int c = lt + kUnpackThreads * i;
+          const bool is_w = c < BW * 4;
+          const int row = (is_w ? c : c - BW * 4) >> 2, cc = c & 3;
+          const uint4 v =
+              *reinterpret_cast<const uint4 *>(pk + (is_w ? 0u : kPackAOff) + row * 64 + cc * 16);
+          uint8_t *dst = op + (is_w ? 0u : kOpAOff) + row * 128;
+          const uint4 lo = make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
+                                      (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
+          const uint4 hi = make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
+                                      v.w & 0xF0F0F0F0u);
+          const int swz = row & 7;
+          *reinterpret_cast<uint4 *>(dst + (((2 * cc) ^ swz) << 4)) = lo;
+          *reinterpret_cast<uint4 *>(dst + (((2 * cc + 1) ^ swz) << 4)) = hi;
+        }
+      } else {
+        // the INT8 group arrived already swizzled: W8 in slot p0, A8 in slot p1
+        const uint8_t *pk1 = pring + p1.idx * kPSlot;
+#pragma unroll
+        for (int i = 0; i < kInt8Chunks / kUnpackThreads; ++i) {
+          const int c = lt + kUnpackThreads * i;
+          const bool is_w = c < BW * 8;
+          const uint32_t off = (is_w ? c : c - BW * 8) * 16u;
+          *reinterpret_cast<uint4 *>(op + (is_w ? 0u : kOpAOff) + off) =
+              *reinterpret_cast<const uint4 *>((is_w ? pk : pk1) + off);
+        }
+      }
+      // scales: sw of the tile's weight rows, and per token pair
+      // (sa'[2j], sa'[2j+1], -C*sa'[2j], -C*sa'[2j+1]) with sa' = sa (times
+      // 1/256 for an INT4 group) truncated to 22 significant bits, the same
+      // fp32 steps as gemm.cuh's drain
+      uint8_t *ss = sring + sl * kSSlot;
+      if (lt < BW) {
+        reinterpret_cast<float *>(ss + kSwOff)[lt] = sc[0];
+      } else if (lt < BW + kMaxTokens / 2) {
+        const int j = lt - BW;
+        float sv[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float s = sc[h];
+          if (int4_group) s *= 0.00390625f;
+          sv[h] = __uint_as_float(__float_as_uint(s) & 0xFFFFFFFCu);
+        }
+        reinterpret_cast<float4 *>(ss)[j] =
+            make_float4(sv[0], sv[1], -gemm_cfg::kBiasF * sv[0], -gemm_cfg::kBiasF * sv[1]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&pempty[p0.idx]);
+        if (!int4_group) mbar_arrive(&pempty[p1.idx]);
+        mbar_arrive(&sfull[sl]);
+        mbar_arrive(&ufull[u]);
+      }
+      pr = p1;
+      if (!int4_group) pr.next(kNP);
+      sc[0] = sc_next[0];
+      sc[1] = sc_next[1];
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+}  // namespace atomk
