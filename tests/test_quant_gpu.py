@@ -34,7 +34,7 @@ def test_weight_codes_bit_exact_all_rows(c_oracle, c):
 
 
 @pytest.mark.parametrize("M,K,seed", [(1, 256, 1), (3, 384, 2), (333, 1152, 3), (777, 4224, 4),
-                                      (64, 32768, 5)])
+                                      (64, 32768, 5), (1000, 24576, 6)])
 def test_ragged_sizes_unsorted_outliers(c_oracle, M, K, seed):
     A, _, idx = inputs.random_case(seed, M, 8, K, dist="t", param=3.0, outlier_factor=50.0,
                                    sorted_outliers=False)

@@ -29,9 +29,6 @@ struct DeviceState {
   bool w8a8_attr = false;
   int w8a8_clusters = 0;          // co-resident CTA pairs of the W8A8 kernel
   uint32_t quant_smem_set = 0;
-  int64_t quant_k = -1;         // K the cached quantizer launch shape is for
-  int quant_stages = 0;         // rows in flight per CTA for that K
-  int quant_occ = 0;            // co-resident quantizer CTAs per SM for that K
   void *noalloc_scratch = nullptr;  // device address of g_noalloc_scratch on this device
 };
 
@@ -87,50 +84,33 @@ atom_status_t launch_quant(const void *x, int64_t rows, int64_t K, int64_t ld,
   DeviceState *dev = nullptr;
   if ((st = current_device(&dev)) != ATOM_OK) return st;
 
-  // Rows in flight per CTA (2 or 3): the choice that keeps the most rows in
-  // flight per SM, and at a tie the one with more CTAs (worked out once per K
-  // and cached).
-  int stages = 0, occ = 0;
+  // One CTA per SM. Its crews share the rows; each crew has its own ring of
+  // 2-4 rows in flight. As many rows as shared memory holds beside the gather
+  // table (at most 12), in as many crews (up to 3) as leave each ring >= 2.
+  const int64_t fixed = atomk::quant_layout(static_cast<int>(K), 0).total;
+  const int64_t row_bytes = 2 * K;
+  int64_t fit = (dev->smem_optin - fixed) / row_bytes;
+  if (fit > atomk::kQuantMaxStages) fit = atomk::kQuantMaxStages;
+  if (fit < 2) return ATOM_ERR_SHAPE;
+  const int64_t crews = fit / 2 < atomk::kQuantCrews ? fit / 2 : atomk::kQuantCrews;
+  const int64_t stages = fit / crews < 4 ? fit / crews : 4;
+  const atomk::QuantLayout L =
+      atomk::quant_layout(static_cast<int>(K), static_cast<int>(stages * crews));
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (dev->quant_k != K) {
-      int best_stages = 0, best_occ = 0;
-      for (int n = 3; n >= 2; --n) {
-        const atomk::QuantLayout l = atomk::quant_layout(static_cast<int>(K), n);
-        if (static_cast<int>(l.total) > dev->smem_optin) continue;
-        if (dev->quant_smem_set < l.total) {
-          if (cudaFuncSetAttribute(atomk::reorder_quant_kernel,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(l.total)) != cudaSuccess)
-            return ATOM_ERR_CUDA;
-          dev->quant_smem_set = l.total;
-        }
-        int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, atomk::reorder_quant_kernel,
-                                                          atomk::kQuantThreads,
-                                                          l.total) != cudaSuccess)
-          return ATOM_ERR_CUDA;
-        // most rows in flight per SM; at a tie, more CTAs (more warps)
-        if (per_sm * n > best_occ * best_stages ||
-            (per_sm * n == best_occ * best_stages && per_sm > best_occ)) {
-          best_occ = per_sm;
-          best_stages = n;
-        }
-      }
-      if (best_stages == 0) return ATOM_ERR_SHAPE;
-      dev->quant_stages = best_stages;
-      dev->quant_occ = best_occ;
-      dev->quant_k = K;
+    if (dev->quant_smem_set < L.total) {
+      if (cudaFuncSetAttribute(atomk::reorder_quant_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(L.total)) != cudaSuccess)
+        return ATOM_ERR_CUDA;
+      dev->quant_smem_set = L.total;
     }
-    stages = dev->quant_stages;
-    occ = dev->quant_occ;
   }
-  const atomk::QuantLayout L = atomk::quant_layout(static_cast<int>(K), stages);
-  const int64_t want = static_cast<int64_t>(occ) * dev->sm_count;
-  const int grid = static_cast<int>(rows < want ? rows : want);
+  const int grid = static_cast<int>(rows < dev->sm_count ? rows : dev->sm_count);
   atomk::reorder_quant_kernel<<<grid, atomk::kQuantThreads, L.total,
                                 reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __half *>(x), rows, static_cast<int>(K), ld, idx, q4, q8, scales, stages);
+      static_cast<const __half *>(x), rows, static_cast<int>(K), ld, idx, q4, q8, scales,
+      static_cast<int>(stages), static_cast<int>(crews));
   return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
 }
 

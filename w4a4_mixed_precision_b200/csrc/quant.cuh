@@ -9,13 +9,18 @@
 //
 // Design (HBM-bound, so the aim is to keep HBM busy with few instructions per
 // element):
-//  * each CTA is persistent over rows r = blockIdx.x + i*gridDim.x; a whole
-//    fp16 row is brought into shared memory by one bulk copy (TMA engine,
-//    mbarrier completion), up to kQuantMaxStages rows in flight per CTA; each
-//    quantizing warp frees a stage through its own arrival on an "empty"
-//    mbarrier, and a ninth warp issues the copy that refills it, so the
-//    quantizing warps never wait for one another while the ring has room;
-//  * at start-up each CTA turns the outlier list into a gather table in shared
+//  * one CTA per SM, persistent over rows r = blockIdx.x + i*gridDim.x. It
+//    runs up to three crews, each of 8 quantizing warps and one copy-issuing
+//    warp with its own ring of 2-4 stage slots: the copy warp takes the CTA's
+//    next row from a counter in shared memory whenever a slot of its ring is
+//    free, tags the slot with the row, and brings the whole fp16 row in with
+//    one bulk copy (TMA engine, mbarrier completion); each quantizing warp
+//    frees a slot through its own arrival on an "empty" mbarrier. A crew the
+//    warp scheduler favours thus takes more rows, and the crews end together;
+//    run as three separate CTAs per SM, with fixed rows each, the last one
+//    ended ~25 % after the first;
+//  * at start-up each CTA (once per SM, shared by its crews) turns the outlier
+//    list into a gather table in shared
 //    memory (uint16 [K]): for every group and lane, the byte offsets inside a
 //    staged row of the 16 channels that lane quantizes, in the lane's gather
 //    order. Reordered position p holds the p-th non-outlier channel for
@@ -37,9 +42,20 @@
 
 namespace atomk {
 
-constexpr int kQuantWarps = 8;                          // quantizing warps
-constexpr int kQuantThreads = 32 * (kQuantWarps + 1);     // + one copy-issuing warp
-constexpr int kQuantMaxStages = 4;
+constexpr int kQuantWarps = 8;                            // quantizing warps per crew
+constexpr int kQuantCrews = 3;                            // crews per CTA, + 1 copy warp each
+constexpr int kQuantThreads = 32 * kQuantCrews * (kQuantWarps + 1);
+constexpr int kQuantMaxStages = 12;
+// Header of the dynamic shared memory (byte offsets).
+constexpr uint32_t kQHdrFull = 0;                            // uint64 [kQuantMaxStages]
+constexpr uint32_t kQHdrEmpty = kQHdrFull + 8 * kQuantMaxStages;
+constexpr uint32_t kQHdrFlags = kQHdrEmpty + 8 * kQuantMaxStages;  // int [2]: bad list, abort
+constexpr uint32_t kQHdrNext = kQHdrFlags + 8;               // int: next row to claim
+constexpr uint32_t kQHdrTags = kQHdrNext + 8;                // int [kQuantMaxStages]: row of each slot
+constexpr uint32_t kQHdrSums = 256;                          // int [32]: block-scan partials
+constexpr uint32_t kQHdrBytes = kQHdrSums + 4 * 32;
+static_assert(kQHdrTags + 4 * kQuantMaxStages <= kQHdrSums, "quantizer header");
+static_assert(kQuantThreads <= 1024, "quantizer block");
 // Gather-table entries are 16-bit byte offsets into a staged fp16 row.
 constexpr int kQuantMaxK = 32768;
 
@@ -53,7 +69,7 @@ struct QuantLayout {
 __host__ __device__ inline QuantLayout quant_layout(int K, int stages_n) {
   QuantLayout L;
   L.row_bytes = 2u * static_cast<uint32_t>(K);
-  L.bitmap = 256;                                                  // after barriers and flags
+  L.bitmap = kQHdrBytes;                                           // after the header
   L.table = L.bitmap + ((static_cast<uint32_t>(K) / 8u + 15u) & ~15u);
   L.stages = (L.table + L.row_bytes + 127u) & ~127u;
   L.stages_n = stages_n;
@@ -82,51 +98,76 @@ __device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t 
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, 1)
 reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t ld,
                      const int32_t *__restrict__ outlier_idx, uint8_t *__restrict__ q4,
-                     int8_t *__restrict__ q8, float *__restrict__ scales, int stages_n) {
+                     int8_t *__restrict__ q8, float *__restrict__ scales, int stages_n,
+                     int crews_n) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  const QuantLayout L = quant_layout(K, stages_n);
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem);                 // [kQuantMaxStages]
-  uint64_t *empty = full + kQuantMaxStages;                            // [kQuantMaxStages]
-  volatile int *flags = reinterpret_cast<volatile int *>(smem + 96);  // [0] bad list, [1] abort
-  int *warp_sums = reinterpret_cast<int *>(smem + 128);               // [8]
+  const QuantLayout L = quant_layout(K, stages_n * crews_n);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kQHdrFull);
+  uint64_t *empty = reinterpret_cast<uint64_t *>(smem + kQHdrEmpty);
+  volatile int *flags = reinterpret_cast<volatile int *>(smem + kQHdrFlags);  // [0] bad list, [1] abort
+  int *next_row = reinterpret_cast<int *>(smem + kQHdrNext);
+  volatile int *tags = reinterpret_cast<volatile int *>(smem + kQHdrTags);
+  int *warp_sums = reinterpret_cast<int *>(smem + kQHdrSums);
   uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem + L.bitmap);
   uint16_t *table = reinterpret_cast<uint16_t *>(smem + L.table);
   uint8_t *stage_base = smem + L.stages;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int crew = warp / (kQuantWarps + 1), cw = warp % (kQuantWarps + 1);
   const int G = K / 128, Gd = G - 1, Kd = K - 128;
   const int64_t q4_row = Kd / 2;
   const int64_t grid = gridDim.x;
+  // this CTA's rows are blockIdx.x + i*grid for i < n_rows (grid <= rows)
+  const int64_t n_rows = (rows - blockIdx.x + grid - 1) / grid;
+  // the outlier list is read once, as early as possible
+  const int oc = tid < 128 ? __ldg(outlier_idx + tid) : 0;
 
   if (tid == 0) {
-    for (int s = 0; s < stages_n; ++s) {
+    for (int s = 0; s < stages_n * crews_n; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kQuantWarps);
     }
     flags[0] = 0;
     flags[1] = 0;
+    *next_row = 0;
     fence_mbar_init();
   }
   for (int w = tid; w < K / 32; w += kQuantThreads) bitmap[w] = 0u;
   __syncthreads();
 
-  // Put the first rows in flight before building the table.
-  if (tid == 0) {
-    for (int s = 0; s < stages_n; ++s) {
-      const int64_t r = blockIdx.x + s * grid;
-      if (r < rows) {
-        mbar_arrive_expect_tx(&full[s], L.row_bytes);
-        bulk_load(stage_base + s * L.row_bytes, x + r * ld, L.row_bytes, &full[s]);
-      }
+  // This crew's ring: stages_n slots with their barriers and row tags.
+  uint64_t *cfull = full + crew * stages_n;
+  uint64_t *cempty = empty + crew * stages_n;
+  volatile int *ctags = tags + crew * stages_n;
+  uint8_t *cstage = stage_base + static_cast<size_t>(crew) * stages_n * L.row_bytes;
+  const bool copier = cw == kQuantWarps && lane == 0 && crew < crews_n;
+  // Takes the CTA's next row for ring slot s and puts it in flight; past the
+  // last row it completes the slot's phase with a plain arrival and a tag
+  // >= n_rows instead, which tells the crew to stop.
+  auto claim = [&](int s) -> bool {
+    const int i = atomicAdd(next_row, 1);
+    ctags[s] = i;
+    if (i >= n_rows) {
+      mbar_arrive(&cfull[s]);
+      return false;
     }
-  }
+    const int64_t r = blockIdx.x + static_cast<int64_t>(i) * grid;
+    mbar_arrive_expect_tx(&cfull[s], L.row_bytes);
+    bulk_load(cstage + s * L.row_bytes, x + r * ld, L.row_bytes, &cfull[s]);
+    return true;
+  };
+  // Each crew's first rows go in flight before the table is built.
+  int issued = 0;
+  bool more = true;
+  if (copier)
+    for (; issued < stages_n && more; ++issued) more = claim(issued);
 
   // ---- gather table: ascending non-outlier channels, then the outlier list.
   if (tid < 128) {
-    const int c = outlier_idx[tid];
+    const int c = oc;
     if (c < 0 || c >= K) {
       flags[0] = 1;
     } else {
@@ -161,58 +202,54 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     }
   }
   if (tid < 128) {
-    const int c = outlier_idx[tid];
+    const int c = oc;
     if (c >= 0 && c < K) table[quant_table_index(Kd + tid, Gd)] = static_cast<uint16_t>(2 * c);
   }
   __syncthreads();
 
   if (flags[0]) {
     // Invalid outlier list: write nothing, but let the issued copies land first.
-    if (tid == 0) {
-      report_status(1 /* ATOM_ERR_INVALID_ARG */);
-      for (int s = 0; s < stages_n; ++s)
-        if (blockIdx.x + s * grid < rows) (void)mbar_wait(&full[s], 0, nullptr);
-    }
+    if (tid == 0) report_status(1 /* ATOM_ERR_INVALID_ARG */);
+    if (copier)
+      for (int s = 0; s < issued; ++s) (void)mbar_wait(&cfull[s], 0, nullptr);
     return;
   }
+  if (crew >= crews_n) return;
 
-  if (warp == kQuantWarps) {
-    // ---- copy issuer: refills each stage slot as soon as all quantizing
-    // warps have released it (slot i % stages_n holds row blockIdx.x + i*grid;
-    // rows 0..stages_n-1 were issued above).
-    if (lane == 0) {
+  if (cw == kQuantWarps) {
+    // ---- copy issuer of this crew: refills each slot of the ring as soon as
+    // the crew's 8 warps have released it, with the CTA's next row.
+    if (copier && more) {
       int sl = 0;
       uint32_t eph = 0;
-      int64_t i = stages_n;
-      for (;; ++i) {
-        const int64_t r = blockIdx.x + i * grid;
-        if (r >= rows) break;
-        if (!mbar_wait(&empty[sl], eph, &flags[1])) {
+      int64_t k = issued;  // ring positions filled so far
+      for (;;) {
+        if (!mbar_wait(&cempty[sl], eph, &flags[1])) {
           if (!flags[1]) report_status(6 /* ATOM_ERR_TIMEOUT */);
           flags[1] = 1;
           break;
         }
-        mbar_arrive_expect_tx(&full[sl], L.row_bytes);
-        bulk_load(stage_base + sl * L.row_bytes, x + r * ld, L.row_bytes, &full[sl]);
+        const bool go = claim(sl);
+        ++k;
         if (++sl == stages_n) {
           sl = 0;
           eph ^= 1u;
         }
+        if (!go) break;
       }
       if (flags[1]) {
         // after an abort, give the copies that may still be in flight (the
         // last one issued into each slot) a bounded chance to land before the
         // CTA's shared memory is released
-        for (int64_t j = (i > stages_n ? i - stages_n : 0); j < i; ++j)
-          if (blockIdx.x + j * grid < rows)
-            (void)mbar_wait(&full[j % stages_n], static_cast<uint32_t>((j / stages_n) & 1), nullptr);
+        for (int64_t j = (k > stages_n ? k - stages_n : 0); j < k; ++j)
+          (void)mbar_wait(&cfull[j % stages_n], static_cast<uint32_t>((j / stages_n) & 1), nullptr);
       }
     }
     return;
   }
 
-  // ---- per-lane constants: group g = pass*32 + 4*warp + team, elements
-  // [16*sub, 16*sub + 16) of the group.
+  // ---- quantizing warps: warp cw of the crew; per-lane constants: group
+  // g = pass*32 + 4*cw + team, elements [16*sub, 16*sub + 16) of the group.
   const int sub = lane & 7;
   const int team = lane >> 3;
   const unsigned team_mask = 0xFFu << (8 * team);
@@ -225,27 +262,28 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     sel_hi |= static_cast<uint32_t>((j + 4 - krot) & 7) << (4 * j);
   }
 
-  // Stage slot and barrier parity of row i, advanced by counting (no
-  // division on the per-row path).
+  // The crew's ring is consumed in order: slot and barrier parity advance by
+  // counting; the slot's tag says which row it holds.
   int s = 0;
   uint32_t ph = 0;
-  for (int64_t i = 0;; ++i) {
-    const int64_t r = blockIdx.x + i * grid;
-    if (r >= rows) break;
-    if (!mbar_wait(&full[s], ph, &flags[1])) {
+  for (;;) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&cfull[s], ph, &flags[1]))) {
       if (lane == 0) {
-        report_status(6 /* ATOM_ERR_TIMEOUT */);
+        if (!flags[1]) report_status(6 /* ATOM_ERR_TIMEOUT */);
         flags[1] = 1;
       }
       break;
     }
-    const uint8_t *row = stage_base + s * L.row_bytes;
+    const int i = ctags[s];
+    if (i >= n_rows) break;
+    const int64_t r = blockIdx.x + static_cast<int64_t>(i) * grid;
+    const uint8_t *row = cstage + s * L.row_bytes;
     uint8_t *q4_r = q4 + r * q4_row;
     int8_t *q8_r = q8 + r * 128;
     float *scales_r = scales + r;
 
     for (int gb = 0; gb < G; gb += 32) {
-      const int g = gb + warp * 4 + team;
+      const int g = gb + cw * 4 + team;
       if (g > Gd) continue;  // whole 8-lane teams skip together
       const bool dense = g < Gd;
       const uint16_t *tb = table + ((g * 2) * 8 + sub) * 8;
@@ -300,7 +338,7 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     }
 
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    if (lane == 0) mbar_arrive(&cempty[s]);
     if (++s == stages_n) {
       s = 0;
       ph ^= 1u;
