@@ -61,7 +61,7 @@ constexpr int kQuantMaxK = 32768;
 
 struct QuantLayout {
   // Byte offsets inside dynamic shared memory.
-  uint32_t bitmap, table, stages, total;
+  uint32_t bitmap, wbase, table, stages, total;
   uint32_t row_bytes;
   int stages_n;
 };
@@ -70,7 +70,8 @@ __host__ __device__ inline QuantLayout quant_layout(int K, int stages_n) {
   QuantLayout L;
   L.row_bytes = 2u * static_cast<uint32_t>(K);
   L.bitmap = kQHdrBytes;                                           // after the header
-  L.table = L.bitmap + ((static_cast<uint32_t>(K) / 8u + 15u) & ~15u);
+  L.wbase = L.bitmap + ((static_cast<uint32_t>(K) / 8u + 15u) & ~15u);   // int [K/32]
+  L.table = L.wbase + ((static_cast<uint32_t>(K) / 8u + 15u) & ~15u);
   L.stages = (L.table + L.row_bytes + 127u) & ~127u;
   L.stages_n = stages_n;
   L.total = L.stages + static_cast<uint32_t>(stages_n) * L.row_bytes;
@@ -112,6 +113,7 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
   volatile int *tags = reinterpret_cast<volatile int *>(smem + kQHdrTags);
   int *warp_sums = reinterpret_cast<int *>(smem + kQHdrSums);
   uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem + L.bitmap);
+  int *wbase = reinterpret_cast<int *>(smem + L.wbase);
   uint16_t *table = reinterpret_cast<uint16_t *>(smem + L.table);
   uint8_t *stage_base = smem + L.stages;
 
@@ -159,11 +161,12 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     bulk_load(cstage + s * L.row_bytes, x + r * ld, L.row_bytes, &cfull[s]);
     return true;
   };
-  // Each crew's first rows go in flight before the table is built.
+  // Each crew's first row goes in flight before the table is built, the rest
+  // of its ring right after: rows all requested at once would land together,
+  // only once the whole burst has been served.
   int issued = 0;
   bool more = true;
-  if (copier)
-    for (; issued < stages_n && more; ++issued) more = claim(issued);
+  if (copier) more = claim(issued++);
 
   // ---- gather table: ascending non-outlier channels, then the outlier list.
   if (tid < 128) {
@@ -191,13 +194,23 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
   __syncthreads();
   int base = 0;
   for (int w = 0; w < warp; ++w) base += warp_sums[w];
-  int pos = base + incl - count;
-  for (int w = w0; w < w1; ++w) {
-    uint32_t bits = ~bitmap[w];
+  // wbase[w]: reordered position of the first non-outlier channel of word w
+  for (int w = w0, p = base + incl - count; w < w1; ++w) {
+    wbase[w] = p;
+    p += __popc(~bitmap[w]);
+  }
+  __syncthreads();
+  // table entries of the non-outlier channels, a quarter word (8 channels) per item
+  for (int it = tid; it < nwords * 4; it += kQuantThreads) {
+    const int w = it >> 2, qtr = it & 3;
+    const uint32_t nb = ~bitmap[w];
+    int pos = wbase[w] + __popc(nb & ((1u << (8 * qtr)) - 1u));
+    uint32_t bits = (nb >> (8 * qtr)) & 0xFFu;
     while (bits) {
       const int b = __ffs(bits) - 1;
       bits &= bits - 1;
-      if (pos < Kd) table[quant_table_index(pos, Gd)] = static_cast<uint16_t>(2 * (w * 32 + b));
+      if (pos < Kd)
+        table[quant_table_index(pos, Gd)] = static_cast<uint16_t>(2 * (w * 32 + 8 * qtr + b));
       ++pos;
     }
   }
@@ -217,8 +230,11 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
   if (crew >= crews_n) return;
 
   if (cw == kQuantWarps) {
-    // ---- copy issuer of this crew: refills each slot of the ring as soon as
-    // the crew's 8 warps have released it, with the CTA's next row.
+    // ---- copy issuer of this crew: fills the rest of the ring, then refills
+    // each slot as soon as the crew's 8 warps have released it, with the
+    // CTA's next row.
+    if (copier)
+      for (; issued < stages_n && more; ++issued) more = claim(issued);
     if (copier && more) {
       int sl = 0;
       uint32_t eph = 0;
