@@ -122,16 +122,21 @@ ATOM_API atom_status_t atom_quant_weights(const void *w, int64_t N, int64_t K, i
  *   qw4, qw8, sw   weight codes/scales as written by atom_quant_weights (N rows).
  *   y              fp16 [M][N] device (output), row-major.
  *   M >= 0, N >= 8 with N % 8 == 0, K as above; n_outlier == group == 128.
- *   workspace      device scratch for shapes whose output tiles would leave most
- *                  CTA pairs idle (small M, e.g. decode): K is then split into up
- *                  to 16 ranges of >= 4 groups, each range's fp32 partial tile is
- *                  written to workspace [splits][M][N], and a second kernel on the
- *                  same stream sums the ranges in order into y. Caller-owned,
- *                  16-byte aligned, at least atom_gemm_workspace_bytes(M, N, K)
- *                  bytes; its contents need no initialisation and are garbage
- *                  afterwards. NULL, or fewer bytes, runs without splitting K
- *                  (same result up to the fp32 summation order). Two calls that
- *                  overlap on the GPU must not share a workspace.
+ *   workspace      device scratch that lets shapes whose output tiles would leave
+ *                  most SMs idle (small M, e.g. decode) split K into ranges, whose
+ *                  fp32 partial tiles are then summed in range order into y. For
+ *                  M > 64 (up to 16 ranges of >= 4 groups) the partial tiles are
+ *                  written to workspace [splits][M][N] and a second kernel on the
+ *                  same stream sums them. For M <= 64 (up to 8 ranges of >= 2
+ *                  groups) the ranges of a weight tile run as one thread-block
+ *                  cluster that sums them in shared memory: the workspace is then
+ *                  only the caller's consent to the split and is not written.
+ *                  Caller-owned, 16-byte aligned, at least
+ *                  atom_gemm_workspace_bytes(M, N, K) bytes; its contents need no
+ *                  initialisation and are garbage afterwards. NULL, or fewer bytes,
+ *                  runs without splitting K (same result up to the fp32 summation
+ *                  order). Two calls that overlap on the GPU must not share a
+ *                  workspace.
  * Pointers qa4, qw4, qa8, qw8, y must be 16-byte aligned; sa, sw 4-byte.
  */
 ATOM_API atom_status_t atom_w4a4_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa,

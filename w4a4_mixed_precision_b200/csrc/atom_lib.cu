@@ -172,15 +172,17 @@ int gemm_splits(int64_t M, int64_t N, int64_t K, int pairs) {
 atom_status_t gemm_pairs(DeviceState *dev, bool pmode, int *pairs);
 
 // K splits of the small-M GEMM (gemm_small.cuh): one 128-row weight tile per
-// CTA, as many K ranges (of at least 2 groups, at most kMaxSplits) as keep
-// every SM busy without a second wave. 1 = no split.
+// CTA, as many K ranges (of at least 2 groups, at most 8: they form one
+// thread-block cluster of portable size) as keep every SM busy without a
+// second wave. 1 = no split.
+constexpr int kMaxSmallSplits = 8;
 int small_splits(int64_t N, int64_t K, int sms) {
   const int64_t n_tiles = (N + atomk::small_cfg::BW - 1) / atomk::small_cfg::BW;
   if (n_tiles <= 0 || n_tiles >= sms) return 1;
   int64_t s = sms / n_tiles;
   const int64_t by_k = (K / 128) / 2;
   if (s > by_k) s = by_k;
-  if (s > kMaxSplits) s = kMaxSplits;
+  if (s > kMaxSmallSplits) s = kMaxSmallSplits;
   return s < 2 ? 1 : static_cast<int>(s);
 }
 
@@ -221,7 +223,6 @@ atom_status_t launch_gemm_small(DeviceState *dev, const uint8_t *qa4, const int8
   p.sa = sa;
   p.sw = sw;
   p.y = static_cast<__half *>(y);
-  p.ws = splits > 1 ? static_cast<float *>(workspace) : nullptr;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
@@ -229,25 +230,29 @@ atom_status_t launch_gemm_small(DeviceState *dev, const uint8_t *qa4, const int8
   p.n_tiles = static_cast<int>((N + BW - 1) / BW);
   p.splits = splits;
   p.items = p.n_tiles * splits;
+  // with a split, one CTA per (tile, K range) and the K ranges of a tile as
+  // one cluster that sums them (no workspace is written)
   const int grid = p.items < dev->sm_count ? p.items : dev->sm_count;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = static_cast<unsigned>(splits);
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaError_t err;
   if (M <= 16)
-    atomk::w4a4_gemm_small_kernel<16><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
+    err = cudaLaunchKernelEx(&cfg, atomk::w4a4_gemm_small_kernel<16>, maps, p);
   else if (M <= 32)
-    atomk::w4a4_gemm_small_kernel<32><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
+    err = cudaLaunchKernelEx(&cfg, atomk::w4a4_gemm_small_kernel<32>, maps, p);
   else
-    atomk::w4a4_gemm_small_kernel<64><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
-  if (cudaGetLastError() != cudaSuccess) return ATOM_ERR_CUDA;
-  if (splits > 1) {
-    const int64_t count8 = M * N / 8;
-    int64_t blocks = (count8 + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(dev->sm_count) * 8;
-    if (blocks > cap) blocks = cap;
-    atomk::splitk_reduce_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
-        p.ws, static_cast<__half *>(y), count8, M * N, splits);
-    if (cudaGetLastError() != cudaSuccess) return ATOM_ERR_CUDA;
-  }
-  return ATOM_OK;
+    err = cudaLaunchKernelEx(&cfg, atomk::w4a4_gemm_small_kernel<64>, maps, p);
+  return err == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
 }
 
 atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa,

@@ -14,8 +14,12 @@
 //   accumulate into an NT-column TMEM accumulator (two alternate); four drain
 //   warps, one per TMEM lane quarter, hold one weight row each and NT token
 //   columns of fp32 accumulators; K is split so that about one CTA per SM
-//   works, each range's fp32 partial tile going to the caller's workspace for
-//   the ordered reduction kernel of gemm.cuh.
+//   works. The K ranges of one weight tile are one thread-block cluster (at
+//   most 8 CTAs): each parks its fp32 partial tile in its own shared memory,
+//   and after a cluster barrier every CTA sums a slice of the tile over all
+//   of them through distributed shared memory, in K-range order, with the
+//   same fp32 additions as the ordered split-K reduction of gemm.cuh, and
+//   writes fp16 Y.
 //
 // Roles (12 warps): warp 0 lane 0 TMA producer; warp 1 lane 0 MMA issuer;
 // warps 2..7 unpack (nibbles to 16*q bytes, K-major, 128-byte swizzle, as in
@@ -69,10 +73,9 @@ struct SmallMaps {
 struct SmallParams {
   const float *sa;   // [G][M]
   const float *sw;   // [G][N]
-  __half *y;         // splits == 1
-  float *ws;         // splits > 1: fp32 partial outputs [splits][M][N]
+  __half *y;
   int M, N, K, G;
-  int n_tiles, splits, items;
+  int n_tiles, splits, items;   // splits > 1: one item per CTA, a cluster of `splits` CTAs per tile
 };
 
 // The (item, group) sequence of one CTA; every role walks the same one. Item i
@@ -238,22 +241,23 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
       }
       if (w.last()) {
         // this K range of the item is complete: write the thread's row of Y
-        // (tokens m < M), or the split's fp32 partial tile; consecutive lanes
-        // write consecutive columns
+        // (tokens m < M); with a split, park the range's fp32 partial tile
+        // [token][weight row] in the operand ring, which no MMA reads any more
+        // (the item is the CTA's only one). Consecutive lanes take consecutive
+        // columns.
         const int n = w.n0 + lrow;
         const bool row_ok = n < p.N;
+        float *part = reinterpret_cast<float *>(uring);
 #pragma unroll
         for (int j = 0; j < NT / 2; ++j) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int m = 2 * j + h;
             const float v = h ? acc[j].y : acc[j].x;
-            if (row_ok && m < p.M) {
-              if (p.splits == 1)
-                p.y[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(v);
-              else
-                p.ws[(static_cast<int64_t>(w.split) * p.M + m) * p.N + n] = v;
-            }
+            if (p.splits > 1)
+              part[m * BW + lrow] = v;
+            else if (row_ok && m < p.M)
+              p.y[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(v);
           }
           acc[j] = make_float2(0.f, 0.f);
         }
@@ -446,6 +450,24 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
   if (warp == 0) {
     tc_fence_after_sync();
     tmem_dealloc(tbase, kTmemCols);
+  }
+  if (p.splits > 1) {
+    // cluster of the tile's K ranges (rank = K range): sum the partial tiles
+    // in range order, a slice of the weight rows per CTA
+    cluster_sync();
+    const int S = p.splits;
+    const int rank = static_cast<int>(cluster_cta_rank());
+    const int n0 = (static_cast<int>(blockIdx.x) / S) * BW;
+    const int lo = rank * BW / S, nr = (rank + 1) * BW / S - lo;
+    const float *part = reinterpret_cast<const float *>(uring);
+    for (int e = threadIdx.x; e < p.M * nr; e += kThreads) {
+      const int m = e / nr, row = lo + (e - m * nr);
+      const float *src = part + m * BW + row;
+      float v = ld_shared_cluster_f32(cluster_map(src, 0));
+      for (int r = 1; r < S; ++r) v += ld_shared_cluster_f32(cluster_map(src, r));
+      if (n0 + row < p.N) p.y[static_cast<int64_t>(m) * p.N + n0 + row] = __float2half_rn(v);
+    }
+    cluster_sync();   // no CTA leaves while a peer may still read its tile
   }
 }
 

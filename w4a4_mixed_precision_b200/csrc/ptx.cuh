@@ -285,6 +285,14 @@ __device__ __forceinline__ uint32_t cluster_map(const void *p, uint32_t rank) {
   return r;
 }
 
+// 32-bit load from the shared memory of any CTA of the cluster (address from
+// cluster_map).
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
 // Arrive on an mbarrier anywhere in the cluster (release at cluster scope).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
