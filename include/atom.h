@@ -161,6 +161,40 @@ ATOM_API atom_status_t atom_w4a4_gemm_partials(const uint8_t *qa4, const int8_t 
                                       int32_t n_outlier, int32_t group, atom_stream_t stream);
 
 /*
+ * atom_w4a4_gemm_quant -- the GEMM of atom_w4a4_gemm with the next layer's
+ * activation quantization fused into its epilogue: instead of fp16 Y it writes
+ * the INT4/INT8 codes and scales that atom_reorder_quant would produce from Y,
+ * with Y's last 128 columns as the outlier channels and no other reorder.
+ *
+ * The pages quantize every activation with its outlier channels moved to the
+ * tail ("Atom: Low-bit Quantization for Efficient and Accurate LLM Serving",
+ * paper summary: activations get a dedicated outlier path). Here that reorder is
+ * assumed to be folded offline into this layer's weight rows (and their order
+ * of output channels), so that Y's columns already come out in the next
+ * layer's reordered order; each 128-column group of a row is then formed and
+ * quantized where it is computed. For every row m and group g of Y's columns:
+ *   yh   = fp16_rn(the value atom_w4a4_gemm writes, unsplit),
+ *   amax = max |yh| over the group, qmax = 7 (g < N/128 - 1) or 127 (last group),
+ *   scale = fl32(amax / qmax), inv = fl32(qmax / amax) (both 0 when amax == 0),
+ *   q    = rint(fl32(yh * inv)), ties to even,
+ * packed as atom_reorder_quant packs them.
+ *
+ *   qa4 ... sw     as for atom_w4a4_gemm; M >= 0, K as there.
+ *   N              Y's columns = the next layer's K: N % 128 == 0, 256 <= N <= 32768.
+ *   qy4            uint8 [M][(N-128)/2] device (output), INT4 codes of groups 0..N/128-2.
+ *   qy8            int8  [M][128] device (output), INT8 codes of Y's last 128 columns.
+ *   sy             float [N/128][M] device (output), group scales.
+ * K is never split (no workspace). qy4 and qy8 must be 16-byte aligned, sy 4-byte.
+ * Errors as atom_w4a4_gemm; ATOM_ERR_SHAPE for an N outside the range above.
+ */
+ATOM_API atom_status_t atom_w4a4_gemm_quant(const uint8_t *qa4, const int8_t *qa8,
+                                           const float *sa, const uint8_t *qw4,
+                                           const int8_t *qw8, const float *sw, int64_t M,
+                                           int64_t N, int64_t K, int32_t n_outlier,
+                                           int32_t group, uint8_t *qy4, int8_t *qy8, float *sy,
+                                           atom_stream_t stream);
+
+/*
  * Bytes of workspace atom_w4a4_gemm uses for this shape on the current device:
  * splits * M * N * 4 when it would split K, else 0 (also 0 on error).
  */

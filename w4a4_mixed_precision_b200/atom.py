@@ -48,6 +48,8 @@ SIGNATURES = {
     "atom_w4a4_gemm_partials": ([ct.c_void_p] * 8 + [ct.c_int64, ct.c_int64, ct.c_int64,
                                                      ct.c_int32, ct.c_int32, ct.c_void_p],
                                 ct.c_int),
+    "atom_w4a4_gemm_quant": ([ct.c_void_p] * 6 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_int32,
+                              ct.c_int32] + [ct.c_void_p] * 4, ct.c_int),
     "atom_gemm_workspace_bytes": ([ct.c_int64, ct.c_int64, ct.c_int64], ct.c_size_t),
     "atom_w4a4_gemm_noalloc": ([ct.c_void_p] * 7 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_int32,
                                                     ct.c_int32, ct.c_void_p], ct.c_int),
@@ -222,6 +224,25 @@ def atom_w4a4_gemm_partials(qa: Quantized, qw: Quantized, K: int,
         M, N, K, N_OUTLIER, GROUP, _stream(stream))
     _check("atom_w4a4_gemm_partials", st)
     return partials, y
+
+
+def atom_w4a4_gemm_quant(qa: Quantized, qw: Quantized, K: int, out: Optional[Quantized] = None,
+                         stream=None) -> Quantized:
+    """The GEMM with the next layer's activation quantization in its epilogue: the codes
+    and scales atom_reorder_quant would write for Y (unsplit, fp16) with Y's last 128
+    columns as the outlier channels (see include/atom.h). N must be a multiple of 128."""
+    M, N = qa.rows, qw.rows
+    if out is None:
+        out = empty_quantized(M, N, qa.q4.device)
+    st = lib().atom_w4a4_gemm_quant(
+        _dev(qa.q4, torch.uint8, "qa4"), _dev(qa.q8, torch.int8, "qa8"),
+        _dev(qa.scales, torch.float32, "sa"), _dev(qw.q4, torch.uint8, "qw4"),
+        _dev(qw.q8, torch.int8, "qw8"), _dev(qw.scales, torch.float32, "sw"),
+        M, N, K, N_OUTLIER, GROUP,
+        _dev(out.q4, torch.uint8, "qy4"), _dev(out.q8, torch.int8, "qy8"),
+        _dev(out.scales, torch.float32, "sy"), _stream(stream))
+    _check("atom_w4a4_gemm_quant", st)
+    return out
 
 
 def atom_w8a8_gemm(qa: torch.Tensor, sa: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor,

@@ -23,8 +23,8 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   int smem_optin = 0;
-  bool gemm_attr[2] = {false, false};
-  int gemm_clusters[2] = {0, 0};  // co-resident CTA pairs of the GEMM kernel
+  bool gemm_attr[3] = {false, false, false};  // by GEMM mode (Y, partials, quantized Y)
+  int gemm_clusters[3] = {0, 0, 0};  // co-resident CTA pairs of the GEMM kernel
   bool small_attr = false;       // shared-memory limit set for the small-M GEMM kernels
   bool w8a8_attr = false;
   int w8a8_clusters = 0;          // co-resident CTA pairs of the W8A8 kernel
@@ -169,7 +169,10 @@ int gemm_splits(int64_t M, int64_t N, int64_t K, int pairs) {
   return s < 2 ? 1 : static_cast<int>(s);
 }
 
-atom_status_t gemm_pairs(DeviceState *dev, bool pmode, int *pairs);
+// Epilogues of the W4A4 GEMM kernel.
+enum GemmMode { kModeY = 0, kModePartials = 1, kModeQuantY = 2 };
+
+atom_status_t gemm_pairs(DeviceState *dev, int mode, int *pairs);
 
 // K splits of the small-M GEMM (gemm_small.cuh): one 128-row weight tile per
 // CTA, as many K ranges (of at least 2 groups, at most 8: they form one
@@ -259,20 +262,26 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
                           const uint8_t *qw4, const int8_t *qw8, const float *sw, void *y,
                           int32_t *partials, int64_t M, int64_t N, int64_t K, int32_t n_outlier,
                           int32_t group, void *workspace, size_t workspace_bytes,
-                          atom_stream_t stream) {
+                          atom_stream_t stream, uint8_t *qy4 = nullptr, int8_t *qy8 = nullptr,
+                          float *sy = nullptr) {
   if (M < 0 || N < 0) return ATOM_ERR_INVALID_ARG;
   atom_status_t st = check_method_params(K, n_outlier, group);
   if (st != ATOM_OK) return st;
   if (N < 8 || N % 8 != 0 || M > INT32_MAX || N > INT32_MAX) return ATOM_ERR_SHAPE;
+  const bool qmode = qy4 != nullptr || qy8 != nullptr || sy != nullptr;
+  // quantized Y: N is the next layer's K (whole groups, the INT8 group last)
+  if (qmode && (N % 128 != 0 || N < 256 || N > kMaxK)) return ATOM_ERR_SHAPE;
   // the kernel addresses each packed INT4 matrix with 32-bit byte offsets
   const int64_t q4_row = (K - 128) / 2;
   if (M * q4_row >= (int64_t(1) << 31) || N * q4_row >= (int64_t(1) << 31)) return ATOM_ERR_SHAPE;
   if (M == 0) return ATOM_OK;
-  if (!qa4 || !qa8 || !sa || !qw4 || !qw8 || !sw || (!y && !partials))
+  if (!qa4 || !qa8 || !sa || !qw4 || !qw8 || !sw || (!y && !partials && !qmode) ||
+      (qmode && (!qy4 || !qy8 || !sy)))
     return ATOM_ERR_INVALID_ARG;
   if (!aligned(qa4, 16) || !aligned(qa8, 16) || !aligned(qw4, 16) || !aligned(qw8, 16) ||
       !aligned(sa, 4) || !aligned(sw, 4) || (y && !aligned(y, 16)) ||
-      (partials && !aligned(partials, 16)))
+      (partials && !aligned(partials, 16)) ||
+      (qmode && (!aligned(qy4, 16) || !aligned(qy8, 16) || !aligned(sy, 4))))
     return ATOM_ERR_ALIGN;
 
   DeviceState *dev = nullptr;
@@ -280,11 +289,12 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
 
   using namespace atomk::gemm_cfg;
   const bool pmode = partials != nullptr;
-  if (!pmode && M <= atomk::small_cfg::kMaxTokens)
+  const int mode = pmode ? kModePartials : (qmode ? kModeQuantY : kModeY);
+  if (mode == kModeY && M <= atomk::small_cfg::kMaxTokens)
     return launch_gemm_small(dev, qa4, qa8, sa, qw4, qw8, sw, y, M, N, K, workspace,
                              workspace_bytes, stream);
   int pairs = 0;
-  if ((st = gemm_pairs(dev, pmode, &pairs)) != ATOM_OK) return st;
+  if ((st = gemm_pairs(dev, mode, &pairs)) != ATOM_OK) return st;
 
   const int64_t G = K / 128;
   atomk::GemmMaps maps;
@@ -318,6 +328,9 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   p.sw = sw;
   p.y = static_cast<__half *>(y);
   p.partials = partials;
+  p.qy4 = qy4;
+  p.qy8 = qy8;
+  p.sy = sy;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
@@ -326,8 +339,8 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   p.m_tiles = static_cast<int>((M + kPairM - 1) / kPairM);
   p.n_tiles = static_cast<int>((N + BN - 1) / BN);
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
-  // Split K only for the output, with a workspace large enough for the partials.
-  int splits = pmode ? 1 : gemm_splits(M, N, K, pairs);
+  // Split K only for fp16 Y, with a workspace large enough for the partials.
+  int splits = mode != kModeY ? 1 : gemm_splits(M, N, K, pairs);
   if (splits > 1 && (workspace == nullptr ||
                      workspace_bytes < static_cast<size_t>(splits) * M * N * sizeof(float) ||
                      !aligned(workspace, 16)))
@@ -340,8 +353,10 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   const int64_t used = p.items < pairs ? p.items : pairs;
   const int grid = static_cast<int>(2 * used);   // CTA pairs (cluster of 2)
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (pmode)
+  if (mode == kModePartials)
     atomk::w4a4_gemm_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
+  else if (mode == kModeQuantY)
+    atomk::w4a4_gemm_kernel<false, true><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
   else
     atomk::w4a4_gemm_kernel<false><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
   if (cudaGetLastError() != cudaSuccess) return ATOM_ERR_CUDA;
@@ -358,12 +373,14 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
 }
 
 // Co-resident CTA pairs of the GEMM kernel on this device (cached per device).
-atom_status_t gemm_pairs(DeviceState *dev, bool pmode, int *pairs) {
+atom_status_t gemm_pairs(DeviceState *dev, int mode, int *pairs) {
   using namespace atomk::gemm_cfg;
-  if (!dev->gemm_attr[pmode]) {
+  if (!dev->gemm_attr[mode]) {
     std::lock_guard<std::mutex> lock(g_mutex);
-    const void *fn = pmode ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<true>)
-                           : reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<false>);
+    const void *fn =
+        mode == kModePartials ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<true>)
+        : mode == kModeQuantY ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<false, true>)
+                              : reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<false>);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess)
       return ATOM_ERR_CUDA;
@@ -381,10 +398,10 @@ atom_status_t gemm_pairs(DeviceState *dev, bool pmode, int *pairs) {
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg) != cudaSuccess || clusters < 1)
       clusters = dev->sm_count / 2;
-    dev->gemm_clusters[pmode] = clusters;
-    dev->gemm_attr[pmode] = true;
+    dev->gemm_clusters[mode] = clusters;
+    dev->gemm_attr[mode] = true;
   }
-  *pairs = dev->gemm_clusters[pmode];
+  *pairs = dev->gemm_clusters[mode];
   return ATOM_OK;
 }
 
@@ -537,6 +554,16 @@ atom_status_t atom_w4a4_gemm_partials(const uint8_t *qa4, const int8_t *qa8, con
                      0, stream);
 }
 
+atom_status_t atom_w4a4_gemm_quant(const uint8_t *qa4, const int8_t *qa8, const float *sa,
+                                   const uint8_t *qw4, const int8_t *qw8, const float *sw,
+                                   int64_t M, int64_t N, int64_t K, int32_t n_outlier,
+                                   int32_t group, uint8_t *qy4, int8_t *qy8, float *sy,
+                                   atom_stream_t stream) {
+  if ((!qy4 || !qy8 || !sy) && M > 0) return ATOM_ERR_INVALID_ARG;
+  return launch_gemm(qa4, qa8, sa, qw4, qw8, sw, nullptr, nullptr, M, N, K, n_outlier, group,
+                     nullptr, 0, stream, qy4, qy8, sy);
+}
+
 size_t atom_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K < 256) return 0;
   DeviceState *dev = nullptr;
@@ -546,7 +573,7 @@ size_t atom_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= atomk::small_cfg::kMaxTokens) {
     splits = small_splits(N, K, dev->sm_count);
   } else {
-    if (gemm_pairs(dev, false, &pairs) != ATOM_OK) return 0;
+    if (gemm_pairs(dev, kModeY, &pairs) != ATOM_OK) return 0;
     splits = gemm_splits(M, N, K, pairs);
   }
   return splits > 1 ? static_cast<size_t>(splits) * M * N * sizeof(float) : 0;
@@ -630,7 +657,7 @@ extern "C" ATOM_API atom_status_t atom_w4a4_gemm_noalloc(
   DeviceState *dev = nullptr;
   if ((st = current_device(&dev)) != ATOM_OK) return st;
   int pairs = 0;
-  if ((st = gemm_pairs(dev, false, &pairs)) != ATOM_OK) return st;
+  if ((st = gemm_pairs(dev, kModeY, &pairs)) != ATOM_OK) return st;
   const int splits = gemm_splits(M, N, K, pairs);
   if (splits > 1 &&
       static_cast<double>(splits) * M * N * sizeof(float) > static_cast<double>(kNoAllocScratchBytes))

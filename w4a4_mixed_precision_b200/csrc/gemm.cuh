@@ -129,8 +129,11 @@ struct GemmParams {
   const float *sa;
   const uint8_t *qw4;
   const float *sw;
-  __half *y;           // may be null in partials mode
+  __half *y;           // may be null in partials mode; null in quant-out mode
   int32_t *partials;   // partials mode only
+  uint8_t *qy4;        // quant-out mode: Y's INT4 codes [M][(N-128)/2],
+  int8_t *qy8;         //   INT8 codes of its last 128 columns [M][128],
+  float *sy;           //   and group scales [N/128][M]
   float *ws;           // splits > 1: fp32 partial outputs [splits][M][N]
   int M, N, K, G;
   int m_tiles, n_tiles, tiles;   // pair tiles of 256 x 256
@@ -319,7 +322,7 @@ struct GemmMaps {
 
 // Hardware barrier ids for the role-internal gathers (0 is __syncthreads).
 
-template <bool kPartials>
+template <bool kPartials, bool kQuantOut = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::kThreads, 1)
 w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   using namespace gemm_cfg;
@@ -497,7 +500,64 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         mbar_arrive(&sempty[sl]);
       }
 
-      if (w.last()) {
+      if constexpr (kQuantOut) {
+        if (w.last()) {
+          // epilogue that writes the next layer's activation codes of Y instead
+          // of Y. This thread's row and 128 columns are one group of Y; Y's
+          // columns are taken to be in the next layer's reordered channel order
+          // already, its last 128 columns being the INT8 outlier group. The
+          // steps are those of the activation quantizer applied to fp16 Y: amax
+          // of the fp16 values, scale = fl(amax/qmax), inv = fl(qmax/amax),
+          // codes = low byte of fl(fl(y*inv) + 1.5*2^23) (round half to even),
+          // element 2i in the low nibble of byte i.
+          const int row = w.m0 + BM * rank + lrow;
+          const int gy = (w.n0 >> 7) + hh;
+          const int Gy = p.N >> 7;
+          const bool in = row < p.M && gy < Gy;
+          const bool dense = gy < Gy - 1;
+          float amax = 0.f;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const float2 f = __half22float2(__floats2half2_rn(acc[i].x, acc[i].y));
+            acc[i] = f;
+            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
+          const float qmax = dense ? 7.f : 127.f;
+          float scale = 0.f, inv = 0.f;
+          if (amax > 0.f) {
+            scale = __fdiv_rn(amax, qmax);
+            inv = __fdiv_rn(qmax, amax);
+          }
+          const int64_t r = in ? row : 0;
+          uint8_t *d4 = p.qy4 + r * static_cast<int64_t>((p.N - 128) >> 1) + (dense && in ? gy : 0) * 64;
+          int8_t *d8 = p.qy8 + r * 128;
+#pragma unroll
+          for (int blk = 0; blk < 4; ++blk) {   // 32 columns: 16 bytes of INT4 or 32 of INT8 codes
+            uint32_t w4[4], w8[8];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t bt[8];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = acc[16 * blk + 4 * c + e];
+                bt[2 * e] = __float_as_uint(__fadd_rn(__fmul_rn(f.x, inv), 12582912.f));
+                bt[2 * e + 1] = __float_as_uint(__fadd_rn(__fmul_rn(f.y, inv), 12582912.f));
+              }
+              const uint32_t ev = low_bytes4(bt[0], bt[2], bt[4], bt[6]);
+              const uint32_t od = low_bytes4(bt[1], bt[3], bt[5], bt[7]);
+              w4[c] = (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
+              w8[2 * c] = low_bytes4(bt[0], bt[1], bt[2], bt[3]);
+              w8[2 * c + 1] = low_bytes4(bt[4], bt[5], bt[6], bt[7]);
+            }
+            st_global_v4_if(d4 + 16 * blk, w4[0], w4[1], w4[2], w4[3], in && dense);
+            st_global_v4_if(d8 + 32 * blk, w8[0], w8[1], w8[2], w8[3], in && !dense);
+            st_global_v4_if(d8 + 32 * blk + 16, w8[4], w8[5], w8[6], w8[7], in && !dense);
+          }
+          if (in) p.sy[static_cast<int64_t>(gy) * p.M + row] = scale;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.f, 0.f);
+        }
+      } else if (w.last()) {
         // epilogue, 8 columns of this thread's row per step. fp16 Y goes out
         // through shared memory and the TMA, 64 columns at a time: each thread
         // writes its row of the warp's 32 x 64 box (128-byte swizzle: 16-byte

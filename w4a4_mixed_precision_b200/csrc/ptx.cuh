@@ -285,6 +285,11 @@ __device__ __forceinline__ uint32_t cluster_map(const void *p, uint32_t rank) {
   return r;
 }
 
+// Low bytes of four 32-bit words, in order, as one word.
+__device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
 // 32-bit load from the shared memory of any CTA of the cluster (address from
 // cluster_map).
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {

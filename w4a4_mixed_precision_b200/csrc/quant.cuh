@@ -94,10 +94,6 @@ __device__ __forceinline__ int quant_table_index(int p, int Gd) {
   return (((g * 2 + (slot >> 3)) * 8 + sub) << 3) + (slot & 7);
 }
 
-// Low bytes of four 32-bit words, in order, as one word.
-__device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
-}
 
 __global__ void __launch_bounds__(kQuantThreads, 1)
 reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t ld,
