@@ -178,6 +178,8 @@ def main():
                     help="skip the fp16 cuBLAS GEMM of the same shape reported beside the result")
     ap.add_argument("--no-w8a8", action="store_true",
                     help="skip the W8A8 comparator GEMM (and torch._int_mm) of the same shape")
+    ap.add_argument("--no-w4a8", action="store_true",
+                    help="skip the W4A8 variant (INT8 activations, the same INT4 weights)")
     ap.add_argument("--no-gemm-quant", action="store_true",
                     help="skip the GEMM with the next layer's quantization in its epilogue")
     ap.add_argument("--no-kv", action="store_true",
@@ -331,6 +333,76 @@ def main():
                "pipelining": "host-to-device copy, compute and device-to-host copy of "
                              "consecutive steps on three streams, two device buffer sets"}
 
+    # The library's own legs run first, before the dense library comparators,
+    # which leave the GPU at its power cap for a while.
+    # -------- the GEMM with the next layer's activation quantization in its epilogue
+    # (atom_w4a4_gemm_quant), against the unfused pair it replaces: the unsplit GEMM
+    # to fp16 Y, then atom_reorder_quant of Y with its last 128 columns as outliers
+    gemm_quant = None
+    if not args.no_gemm_quant and w.N % 128 == 0 and w.N >= 256:
+        out_f = atom.empty_quantized(w.M, w.N, dev)
+        out_u = atom.empty_quantized(w.M, w.N, dev)
+        y_u = torch.empty((w.M, w.N), dtype=torch.float16, device=dev)
+        tail = torch.arange(w.N - 128, w.N, dtype=torch.int32, device=dev)
+        n_gq = max(3, min(10, n_steps // 20))
+
+        def time_gq(fn):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(n_gq):
+                fn()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            return a0.elapsed_time(a1) / n_gq
+
+        def unfused():
+            atom.atom_w4a4_gemm(qa, qw, w.K, y=y_u, stream=stream, split=False)
+            atom.atom_reorder_quant(y_u, tail, out=out_u, stream=stream)
+
+        f_ms = time_gq(lambda: atom.atom_w4a4_gemm_quant(qa, qw, w.K, out=out_f, stream=stream))
+        u_ms = time_gq(unfused)
+        ops = 2.0 * w.M * w.N * w.K
+        gemm_quant = {"value": round(ops / (f_ms * 1e-3) / 1e12, 2), "unit": "TOPS",
+                      "ms": round(f_ms, 4), "steps": n_gq,
+                      "unfused_ms": round(u_ms, 4),
+                      "output_bytes": w.M * ((w.N - 128) // 2 + 128 + 4 * (w.N // 128)),
+                      "unfused_output_bytes": w.M * w.N * 2,
+                      "kind": "atom_w4a4_gemm_quant: the same GEMM writing the next layer's "
+                              "INT4/INT8 codes and scales of Y instead of fp16 Y; unfused = "
+                              "atom_w4a4_gemm (no K split) then atom_reorder_quant of Y"}
+        del out_f, out_u, y_u
+        if atom.atom_device_status(clear=True) != 0:
+            raise RuntimeError("device status set by the quantizing GEMM")
+
+    # -------- W4A8 variant: INT8 activations in every group, the same INT4 weights
+    w4a8 = None
+    if not args.no_w4a8:
+        qa_a8 = atom.atom_reorder_quant_a8(A, idx, stream=stream)
+        y_a8 = torch.empty((w.M, w.N), dtype=torch.float16, device=dev)
+        n_a8 = max(3, min(10, n_steps // 20))
+        for _ in range(3):
+            atom.atom_w4a8_gemm(qa_a8, qw, w.K, y=y_a8, stream=stream)
+        torch.cuda.synchronize()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n_a8):
+            atom.atom_w4a8_gemm(qa_a8, qw, w.K, y=y_a8, stream=stream)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        a8_ms = a0.elapsed_time(a1) / n_a8
+        w4a8 = {"value": round(2.0 * w.M * w.N * w.K / (a8_ms * 1e-3) / 1e12, 2), "unit": "TOPS",
+                "ms": round(a8_ms, 4), "steps": n_a8,
+                "kind": "atom_w4a8_gemm: INT8 activations (atom_reorder_quant_a8 of the same A) "
+                        "x the same INT4/INT8 weights, fp16 out, no K split"}
+        del qa_a8, y_a8
+        if atom.atom_device_status(clear=True) != 0:
+            raise RuntimeError("device status set by the W4A8 variant")
+
     # -------- fp16 cuBLAS GEMM of the same shape (torch.matmul), a library baseline
     cublas = None
     if not args.no_cublas:
@@ -392,49 +464,6 @@ def main():
         del qa8, qw8, y8
         if atom.atom_device_status(clear=True) != 0:
             raise RuntimeError("device status set by the W8A8 comparator")
-
-    # -------- the GEMM with the next layer's activation quantization in its epilogue
-    # (atom_w4a4_gemm_quant), against the unfused pair it replaces: the unsplit GEMM
-    # to fp16 Y, then atom_reorder_quant of Y with its last 128 columns as outliers
-    gemm_quant = None
-    if not args.no_gemm_quant and w.N % 128 == 0 and w.N >= 256:
-        out_f = atom.empty_quantized(w.M, w.N, dev)
-        out_u = atom.empty_quantized(w.M, w.N, dev)
-        y_u = torch.empty((w.M, w.N), dtype=torch.float16, device=dev)
-        tail = torch.arange(w.N - 128, w.N, dtype=torch.int32, device=dev)
-        n_gq = max(3, min(10, n_steps // 20))
-
-        def time_gq(fn):
-            for _ in range(3):
-                fn()
-            torch.cuda.synchronize()
-            a0 = torch.cuda.Event(enable_timing=True)
-            a1 = torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            for _ in range(n_gq):
-                fn()
-            a1.record(stream)
-            torch.cuda.synchronize()
-            return a0.elapsed_time(a1) / n_gq
-
-        def unfused():
-            atom.atom_w4a4_gemm(qa, qw, w.K, y=y_u, stream=stream, split=False)
-            atom.atom_reorder_quant(y_u, tail, out=out_u, stream=stream)
-
-        f_ms = time_gq(lambda: atom.atom_w4a4_gemm_quant(qa, qw, w.K, out=out_f, stream=stream))
-        u_ms = time_gq(unfused)
-        ops = 2.0 * w.M * w.N * w.K
-        gemm_quant = {"value": round(ops / (f_ms * 1e-3) / 1e12, 2), "unit": "TOPS",
-                      "ms": round(f_ms, 4), "steps": n_gq,
-                      "unfused_ms": round(u_ms, 4),
-                      "output_bytes": w.M * ((w.N - 128) // 2 + 128 + 4 * (w.N // 128)),
-                      "unfused_output_bytes": w.M * w.N * 2,
-                      "kind": "atom_w4a4_gemm_quant: the same GEMM writing the next layer's "
-                              "INT4/INT8 codes and scales of Y instead of fp16 Y; unfused = "
-                              "atom_w4a4_gemm (no K split) then atom_reorder_quant of Y"}
-        del out_f, out_u, y_u
-        if atom.atom_device_status(clear=True) != 0:
-            raise RuntimeError("device status set by the quantizing GEMM")
 
     # -------- INT4 KV cache: 131072 tokens x 8 KV heads x head_dim 128 (268 MB fp16)
     kv = None
@@ -549,6 +578,8 @@ def main():
         line["w8a8"] = w8a8
     if gemm_quant is not None:
         line["gemm_quant"] = gemm_quant
+    if w4a8 is not None:
+        line["w4a8"] = w4a8
     if kv is not None:
         kv["quant"]["frac_hbm"] = round(kv["quant"]["value"] / peaks["hbm_gbs"], 4)
         kv["dequant"]["frac_hbm"] = round(kv["dequant"]["value"] / peaks["hbm_gbs"], 4)

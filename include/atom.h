@@ -161,6 +161,53 @@ ATOM_API atom_status_t atom_w4a4_gemm_partials(const uint8_t *qa4, const int8_t 
                                       int32_t n_outlier, int32_t group, atom_stream_t stream);
 
 /*
+ * W4A8 variant: INT8 activations in every group, the W4A4 weights unchanged.
+ *
+ * The pages set Atom's 4-bit kernels beside 8-bit activation schemes ("Atom:
+ * Low-bit Quantization for Efficient and Accurate LLM Serving", abstract and
+ * paper summary). This variant keeps Atom's layout and outlier reorder, and
+ * quantizes every 128-channel group of the reordered activation row to INT8 with
+ * the same steps as the outlier group ("Atom (mixed-precision block-outlier
+ * low-bit quantization for serving)", fields Weight group size and notes):
+ *   scale = fl32(amax/127), inv = fl32(127/amax) (0 for a zero group),
+ *   q = rint(fl32(x*inv)), ties to even.
+ *
+ * atom_reorder_quant_a8: x, M, K, ld_x, outlier_idx, n_outlier, group as for
+ *   atom_reorder_quant;
+ *   q8      int8 [M][K] device (output), the codes in reordered channel order;
+ *   scales  float [K/128][M] device (output).
+ *   q8 must be 16-byte aligned; errors as atom_reorder_quant.
+ */
+ATOM_API atom_status_t atom_reorder_quant_a8(const void *x, int64_t M, int64_t K, int64_t ld_x,
+                                            const int32_t *outlier_idx, int32_t n_outlier,
+                                            int32_t group, int8_t *q8, float *scales,
+                                            atom_stream_t stream);
+
+/*
+ * atom_w4a8_gemm: Y[m][n] = fp16( sum_g sa[g][m] * sw[g][n] * P[g][m][n] ) with
+ * P[g][m][n] = sum_{k in g} qa8[m][k] * qw[n][k] exact in int32 (INT8 x INT4 for
+ * the dense groups, INT8 x INT8 for the outlier group); fp32 accumulation of
+ * the dequantized partials.
+ *   qa8, sa        as written by atom_reorder_quant_a8 (M rows).
+ *   qw4, qw8, sw   as written by atom_quant_weights (N rows).
+ *   y              fp16 [M][N] device (output).
+ *   M >= 0, N >= 8 with N % 8 == 0, K as for atom_w4a4_gemm. K is never split.
+ * atom_w4a8_gemm_partials: the same, writing P as int32 [G][M][N] (debug) and,
+ *   when y is not NULL, Y.
+ * qa8, qw4, qw8, y, partials must be 16-byte aligned; sa, sw 4-byte.
+ */
+ATOM_API atom_status_t atom_w4a8_gemm(const int8_t *qa8, const float *sa, const uint8_t *qw4,
+                                     const int8_t *qw8, const float *sw, void *y, int64_t M,
+                                     int64_t N, int64_t K, int32_t n_outlier, int32_t group,
+                                     atom_stream_t stream);
+ATOM_API atom_status_t atom_w4a8_gemm_partials(const int8_t *qa8, const float *sa,
+                                              const uint8_t *qw4, const int8_t *qw8,
+                                              const float *sw, int32_t *partials, void *y,
+                                              int64_t M, int64_t N, int64_t K,
+                                              int32_t n_outlier, int32_t group,
+                                              atom_stream_t stream);
+
+/*
  * atom_w4a4_gemm_quant -- the GEMM of atom_w4a4_gemm with the next layer's
  * activation quantization fused into its epilogue: instead of fp16 Y it writes
  * the INT4/INT8 codes and scales that atom_reorder_quant would produce from Y,

@@ -39,6 +39,14 @@ SIGNATURES = {
     "atom_reorder_quant": ([ct.c_void_p, ct.c_int64, ct.c_int64, ct.c_int64, ct.c_void_p,
                             ct.c_int32, ct.c_int32, ct.c_void_p, ct.c_void_p, ct.c_void_p,
                             ct.c_void_p], ct.c_int),
+    "atom_reorder_quant_a8": ([ct.c_void_p, ct.c_int64, ct.c_int64, ct.c_int64, ct.c_void_p,
+                               ct.c_int32, ct.c_int32, ct.c_void_p, ct.c_void_p, ct.c_void_p],
+                              ct.c_int),
+    "atom_w4a8_gemm": ([ct.c_void_p] * 6 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_int32,
+                                            ct.c_int32, ct.c_void_p], ct.c_int),
+    "atom_w4a8_gemm_partials": ([ct.c_void_p] * 7 + [ct.c_int64, ct.c_int64, ct.c_int64,
+                                                     ct.c_int32, ct.c_int32, ct.c_void_p],
+                                ct.c_int),
     "atom_quant_weights": ([ct.c_void_p, ct.c_int64, ct.c_int64, ct.c_int64, ct.c_void_p,
                             ct.c_int32, ct.c_int32, ct.c_void_p, ct.c_void_p, ct.c_void_p,
                             ct.c_void_p], ct.c_int),
@@ -148,6 +156,63 @@ def atom_reorder_quant(x: torch.Tensor, outlier_idx: torch.Tensor,
                        out: Optional[Quantized] = None, stream=None) -> Quantized:
     """Fused outlier reorder + INT4/INT8 quantization of fp16 activations [M, K]."""
     return _quant("atom_reorder_quant", x, outlier_idx, out, stream)
+
+
+class QuantizedA8(NamedTuple):
+    """W4A8 activations: INT8 codes [rows, K] in reordered order, scales [K/128, rows]."""
+    q8: torch.Tensor
+    scales: torch.Tensor
+
+    @property
+    def rows(self) -> int:
+        return self.q8.shape[0]
+
+
+def atom_reorder_quant_a8(x: torch.Tensor, outlier_idx: torch.Tensor,
+                          out: Optional[QuantizedA8] = None, stream=None) -> QuantizedA8:
+    """W4A8 activations: the outlier reorder, then INT8 in every group (see include/atom.h)."""
+    if x.dim() != 2 or x.stride(1) != 1 or not x.is_cuda or x.dtype != torch.float16:
+        raise ValueError("input must be a 2-D CUDA float16 tensor with contiguous rows")
+    rows, K = x.shape
+    if out is None:
+        out = QuantizedA8(torch.empty((rows, K), dtype=torch.int8, device=x.device),
+                          torch.empty((K // GROUP, rows), dtype=torch.float32, device=x.device))
+    st = lib().atom_reorder_quant_a8(x.data_ptr(), rows, K, x.stride(0),
+                                     _dev(outlier_idx, torch.int32, "outlier_idx"),
+                                     outlier_idx.numel(), GROUP, _dev(out.q8, torch.int8, "q8"),
+                                     _dev(out.scales, torch.float32, "scales"), _stream(stream))
+    _check("atom_reorder_quant_a8", st)
+    return out
+
+
+def atom_w4a8_gemm(qa: QuantizedA8, qw: Quantized, K: int, y: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """W4A8: Y fp16 [M, N] from INT8 activations and the W4A4 weights (see include/atom.h)."""
+    M, N = qa.rows, qw.rows
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=qa.q8.device)
+    st = lib().atom_w4a8_gemm(
+        _dev(qa.q8, torch.int8, "qa8"), _dev(qa.scales, torch.float32, "sa"),
+        _dev(qw.q4, torch.uint8, "qw4"), _dev(qw.q8, torch.int8, "qw8"),
+        _dev(qw.scales, torch.float32, "sw"), _dev(y, torch.float16, "y"),
+        M, N, K, N_OUTLIER, GROUP, _stream(stream))
+    _check("atom_w4a8_gemm", st)
+    return y
+
+
+def atom_w4a8_gemm_partials(qa: QuantizedA8, qw: Quantized, K: int, stream=None):
+    """Debug entry of the W4A8 GEMM: per-group int32 partial sums [G, M, N] and Y."""
+    M, N = qa.rows, qw.rows
+    dev = qa.q8.device
+    partials = torch.empty((K // GROUP, M, N), dtype=torch.int32, device=dev)
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    st = lib().atom_w4a8_gemm_partials(
+        _dev(qa.q8, torch.int8, "qa8"), _dev(qa.scales, torch.float32, "sa"),
+        _dev(qw.q4, torch.uint8, "qw4"), _dev(qw.q8, torch.int8, "qw8"),
+        _dev(qw.scales, torch.float32, "sw"), _dev(partials, torch.int32, "partials"),
+        _dev(y, torch.float16, "y"), M, N, K, N_OUTLIER, GROUP, _stream(stream))
+    _check("atom_w4a8_gemm_partials", st)
+    return partials, y
 
 
 def atom_quant_weights(w: torch.Tensor, outlier_idx: torch.Tensor,

@@ -23,8 +23,8 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   int smem_optin = 0;
-  bool gemm_attr[3] = {false, false, false};  // by GEMM mode (Y, partials, quantized Y)
-  int gemm_clusters[3] = {0, 0, 0};  // co-resident CTA pairs of the GEMM kernel
+  bool gemm_attr[6] = {};        // by GEMM kernel: mode (Y, partials, quantized Y) + 3 * W4A8
+  int gemm_clusters[6] = {};     // co-resident CTA pairs of the GEMM kernel
   bool small_attr = false;       // shared-memory limit set for the small-M GEMM kernels
   bool w8a8_attr = false;
   int w8a8_clusters = 0;          // co-resident CTA pairs of the W8A8 kernel
@@ -70,14 +70,14 @@ atom_status_t check_method_params(int64_t K, int32_t n_outlier, int32_t group) {
 
 atom_status_t launch_quant(const void *x, int64_t rows, int64_t K, int64_t ld,
                            const int32_t *idx, int32_t n_outlier, int32_t group, uint8_t *q4,
-                           int8_t *q8, float *scales, atom_stream_t stream) {
+                           int8_t *q8, float *scales, atom_stream_t stream, bool a8 = false) {
   if (rows < 0 || ld < 0) return ATOM_ERR_INVALID_ARG;
   atom_status_t st = check_method_params(K, n_outlier, group);
   if (st != ATOM_OK) return st;
   if (ld < K || ld % 8 != 0) return ATOM_ERR_SHAPE;
   if (rows == 0) return ATOM_OK;
-  if (!x || !idx || !q4 || !q8 || !scales) return ATOM_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(q4, 16) || !aligned(q8, 16) || !aligned(scales, 4) ||
+  if (!x || !idx || (!q4 && !a8) || !q8 || !scales) return ATOM_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || (!a8 && !aligned(q4, 16)) || !aligned(q8, 16) || !aligned(scales, 4) ||
       !aligned(idx, 4))
     return ATOM_ERR_ALIGN;
 
@@ -110,7 +110,7 @@ atom_status_t launch_quant(const void *x, int64_t rows, int64_t K, int64_t ld,
   atomk::reorder_quant_kernel<<<grid, atomk::kQuantThreads, L.total,
                                 reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const __half *>(x), rows, static_cast<int>(K), ld, idx, q4, q8, scales,
-      static_cast<int>(stages), static_cast<int>(crews));
+      static_cast<int>(stages), static_cast<int>(crews), a8 ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
 }
 
@@ -172,7 +172,7 @@ int gemm_splits(int64_t M, int64_t N, int64_t K, int pairs) {
 // Epilogues of the W4A4 GEMM kernel.
 enum GemmMode { kModeY = 0, kModePartials = 1, kModeQuantY = 2 };
 
-atom_status_t gemm_pairs(DeviceState *dev, int mode, int *pairs);
+atom_status_t gemm_pairs(DeviceState *dev, int mode, int *pairs);   // mode + 3 for W4A8
 
 // K splits of the small-M GEMM (gemm_small.cuh): one 128-row weight tile per
 // CTA, as many K ranges (of at least 2 groups, at most 8: they form one
@@ -263,7 +263,7 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
                           int32_t *partials, int64_t M, int64_t N, int64_t K, int32_t n_outlier,
                           int32_t group, void *workspace, size_t workspace_bytes,
                           atom_stream_t stream, uint8_t *qy4 = nullptr, int8_t *qy8 = nullptr,
-                          float *sy = nullptr) {
+                          float *sy = nullptr, bool a8 = false) {
   if (M < 0 || N < 0) return ATOM_ERR_INVALID_ARG;
   atom_status_t st = check_method_params(K, n_outlier, group);
   if (st != ATOM_OK) return st;
@@ -275,11 +275,11 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   const int64_t q4_row = (K - 128) / 2;
   if (M * q4_row >= (int64_t(1) << 31) || N * q4_row >= (int64_t(1) << 31)) return ATOM_ERR_SHAPE;
   if (M == 0) return ATOM_OK;
-  if (!qa4 || !qa8 || !sa || !qw4 || !qw8 || !sw || (!y && !partials && !qmode) ||
+  if ((!qa4 && !a8) || !qa8 || !sa || !qw4 || !qw8 || !sw || (!y && !partials && !qmode) ||
       (qmode && (!qy4 || !qy8 || !sy)))
     return ATOM_ERR_INVALID_ARG;
-  if (!aligned(qa4, 16) || !aligned(qa8, 16) || !aligned(qw4, 16) || !aligned(qw8, 16) ||
-      !aligned(sa, 4) || !aligned(sw, 4) || (y && !aligned(y, 16)) ||
+  if ((!a8 && !aligned(qa4, 16)) || !aligned(qa8, 16) || !aligned(qw4, 16) ||
+      !aligned(qw8, 16) || !aligned(sa, 4) || !aligned(sw, 4) || (y && !aligned(y, 16)) ||
       (partials && !aligned(partials, 16)) ||
       (qmode && (!aligned(qy4, 16) || !aligned(qy8, 16) || !aligned(sy, 4))))
     return ATOM_ERR_ALIGN;
@@ -290,20 +290,23 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   using namespace atomk::gemm_cfg;
   const bool pmode = partials != nullptr;
   const int mode = pmode ? kModePartials : (qmode ? kModeQuantY : kModeY);
-  if (mode == kModeY && M <= atomk::small_cfg::kMaxTokens)
+  if (mode == kModeY && !a8 && M <= atomk::small_cfg::kMaxTokens)
     return launch_gemm_small(dev, qa4, qa8, sa, qw4, qw8, sw, y, M, N, K, workspace,
                              workspace_bytes, stream);
   int pairs = 0;
-  if ((st = gemm_pairs(dev, mode, &pairs)) != ATOM_OK) return st;
+  if ((st = gemm_pairs(dev, mode + (a8 ? 3 : 0), &pairs)) != ATOM_OK) return st;
 
   const int64_t G = K / 128;
   atomk::GemmMaps maps;
   const bool sa_by_tma = (M % 4) == 0;   // rows of sa must be 16-byte aligned for TMA
   const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  if (!encode_2d(&maps.a4, u8, qa4, q4_row, M, q4_row, 64, BM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+  // W4A8: INT8 activations [M][K], one 128-byte box per row and group; no INT4 A
+  if (!encode_2d(&maps.a4, u8, a8 ? static_cast<const void *>(qa8) : qa4, q4_row, M, q4_row, 64,
+                 BM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !encode_2d(&maps.w4, u8, qw4, q4_row, N, q4_row, 64, BW, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_2d(&maps.a8, u8, qa8, 128, M, 128, 128, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&maps.a8, u8, qa8, a8 ? K : 128, M, a8 ? K : 128, 128, BM,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&maps.w8, u8, qw8, 128, N, 128, 128, BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&maps.sw, f32, sw, N, G, N * 4, BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
     return ATOM_ERR_CUDA;
@@ -340,7 +343,7 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   p.n_tiles = static_cast<int>((N + BN - 1) / BN);
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
   // Split K only for fp16 Y, with a workspace large enough for the partials.
-  int splits = mode != kModeY ? 1 : gemm_splits(M, N, K, pairs);
+  int splits = (mode != kModeY || a8) ? 1 : gemm_splits(M, N, K, pairs);
   if (splits > 1 && (workspace == nullptr ||
                      workspace_bytes < static_cast<size_t>(splits) * M * N * sizeof(float) ||
                      !aligned(workspace, 16)))
@@ -353,7 +356,11 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   const int64_t used = p.items < pairs ? p.items : pairs;
   const int grid = static_cast<int>(2 * used);   // CTA pairs (cluster of 2)
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (mode == kModePartials)
+  if (a8 && mode == kModePartials)
+    atomk::w4a4_gemm_kernel<true, false, true><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
+  else if (a8)
+    atomk::w4a4_gemm_kernel<false, false, true><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
+  else if (mode == kModePartials)
     atomk::w4a4_gemm_kernel<true><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
   else if (mode == kModeQuantY)
     atomk::w4a4_gemm_kernel<false, true><<<grid, kThreads, kSmemBytes, s>>>(maps, p);
@@ -380,7 +387,11 @@ atom_status_t gemm_pairs(DeviceState *dev, int mode, int *pairs) {
     const void *fn =
         mode == kModePartials ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<true>)
         : mode == kModeQuantY ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<false, true>)
-                              : reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<false>);
+        : mode == kModeY + 3
+            ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<false, false, true>)
+        : mode == kModePartials + 3
+            ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<true, false, true>)
+            : reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<false>);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess)
       return ATOM_ERR_CUDA;
@@ -552,6 +563,30 @@ atom_status_t atom_w4a4_gemm_partials(const uint8_t *qa4, const int8_t *qa8, con
   if (!partials && M > 0) return ATOM_ERR_INVALID_ARG;
   return launch_gemm(qa4, qa8, sa, qw4, qw8, sw, y, partials, M, N, K, n_outlier, group, nullptr,
                      0, stream);
+}
+
+atom_status_t atom_reorder_quant_a8(const void *x, int64_t M, int64_t K, int64_t ld_x,
+                                    const int32_t *outlier_idx, int32_t n_outlier, int32_t group,
+                                    int8_t *q8, float *scales, atom_stream_t stream) {
+  return launch_quant(x, M, K, ld_x, outlier_idx, n_outlier, group, nullptr, q8, scales, stream,
+                      true);
+}
+
+atom_status_t atom_w4a8_gemm(const int8_t *qa8, const float *sa, const uint8_t *qw4,
+                             const int8_t *qw8, const float *sw, void *y, int64_t M, int64_t N,
+                             int64_t K, int32_t n_outlier, int32_t group, atom_stream_t stream) {
+  if (!y && M > 0) return ATOM_ERR_INVALID_ARG;
+  return launch_gemm(nullptr, qa8, sa, qw4, qw8, sw, y, nullptr, M, N, K, n_outlier, group,
+                     nullptr, 0, stream, nullptr, nullptr, nullptr, true);
+}
+
+atom_status_t atom_w4a8_gemm_partials(const int8_t *qa8, const float *sa, const uint8_t *qw4,
+                                      const int8_t *qw8, const float *sw, int32_t *partials,
+                                      void *y, int64_t M, int64_t N, int64_t K,
+                                      int32_t n_outlier, int32_t group, atom_stream_t stream) {
+  if (!partials && M > 0) return ATOM_ERR_INVALID_ARG;
+  return launch_gemm(nullptr, qa8, sa, qw4, qw8, sw, y, partials, M, N, K, n_outlier, group,
+                     nullptr, 0, stream, nullptr, nullptr, nullptr, true);
 }
 
 atom_status_t atom_w4a4_gemm_quant(const uint8_t *qa4, const int8_t *qa8, const float *sa,

@@ -278,6 +278,40 @@ __device__ __forceinline__ void copy_int8(int lt, const uint8_t *pk_a, const uin
   }
 }
 
+// A W4A8 INT4 group: the INT8 activation tile arrived already in the swizzled
+// MMA layout (`pk_a`) and is copied; the packed INT4 weight tile (`pk_w`, 128
+// rows x 64 bytes) is unpacked to bytes holding 16*q. Unlike unpack_int4, which
+// writes a chunk's even elements before its odd ones (harmless there: A and W
+// share that order), the elements keep their natural K order here, to match A.
+__device__ __forceinline__ void copy_a8_unpack_w4(int lt, const uint8_t *pk_a, const uint8_t *pk_w,
+                                                  uint8_t *op) {
+  using namespace gemm_cfg;
+  constexpr int kAChunks = static_cast<int>(kABytes / 16);
+  for (int c = lt; c < kAChunks + BW * 4; c += kUnpackThreads) {
+    if (c < kAChunks) {
+      *reinterpret_cast<uint4 *>(op + c * 16u) = *reinterpret_cast<const uint4 *>(pk_a + c * 16u);
+    } else {
+      const int cw = c - kAChunks, row = cw >> 2, cc = cw & 3;
+      const uint4 v = *reinterpret_cast<const uint4 *>(pk_w + row * 64 + cc * 16);
+      uint8_t *dst = op + kABytes + row * 128;
+      // packed byte i holds elements 2i (low nibble) and 2i+1: L byte i = 16*q[2i],
+      // H byte i = 16*q[2i+1]; interleave them back into element order
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t L = (w[j] << 4) & 0xF0F0F0F0u, H = w[j] & 0xF0F0F0F0u;
+        o[2 * j] = __byte_perm(L, H, 0x5140);       // elements 8j .. 8j+3
+        o[2 * j + 1] = __byte_perm(L, H, 0x7362);   // elements 8j+4 .. 8j+7
+      }
+      const int sw = row & 7;
+      *reinterpret_cast<uint4 *>(dst + (((2 * cc) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<uint4 *>(dst + (((2 * cc + 1) ^ sw) << 4)) =
+          make_uint4(o[4], o[5], o[6], o[7]);
+    }
+  }
+}
+
 // Lays the group's scales out for the drain (threads 0..127: sa; 128..191: sw).
 // `sa_direct` is this thread's sa value when sa does not come through TMA.
 __device__ __forceinline__ void layout_scales(const GemmParams &p, int lt, const uint8_t *pk,
@@ -322,7 +356,9 @@ struct GemmMaps {
 
 // Hardware barrier ids for the role-internal gathers (0 is __syncthreads).
 
-template <bool kPartials, bool kQuantOut = false>
+// kA8: W4A8, the activations are INT8 in every group ([M][K], loaded per
+// group like the INT8 outlier tile); the INT4 weight groups unpack as usual.
+template <bool kPartials, bool kQuantOut = false, bool kA8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_cfg::kThreads, 1)
 w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   using namespace gemm_cfg;
@@ -439,7 +475,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       // 1/256 for the INT4 groups, whose partials are 256*P) truncated to 22
       // significant bits so that C*sa' is exact; then acc += t * sw.
       float sa = reinterpret_cast<const float *>(ss)[lrow];
-      if (w.g < p.G - 1) sa *= 0.00390625f;
+      if (w.g < p.G - 1) sa *= kA8 ? 0.0625f : 0.00390625f;
       sa = __uint_as_float(__float_as_uint(sa) & 0xFFFFFFFCu);
       const float2 sa2 = make_float2(sa, sa);
       const float2 nc2 = make_float2(-kBiasF * sa, -kBiasF * sa);
@@ -459,7 +495,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
           // wholly inside or wholly outside the matrix.
           const int row = w.m0 + BM * rank + lrow;
           const int col0 = w.n0 + hh * kHalfN + 16 * c;
-          const int sh = w.g < p.G - 1 ? 8 : 0;
+          const int sh = w.g < p.G - 1 ? (kA8 ? 4 : 8) : 0;
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             const int col = col0 + 4 * v;
@@ -615,7 +651,8 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         for (int64_t it = 0; ok && it < iters; ++it, wp.next(p)) {
           const int arow = wp.m0 + BM * rank, wrow = wp.n0 + BW * rank;
           const bool int4_group = wp.g < p.G - 1;
-          for (int part = 0; part < (int4_group ? 1 : 2); ++part) {
+          const bool two_slots = kA8 || !int4_group;   // INT8 A tile in its own slot
+          for (int part = 0; part < (two_slots ? 2 : 1); ++part) {
             const int s = pr.idx;
             if (!mbar_wait(&pempty[s], pr.phase ^ 1u, abort_flag)) {
               ok = false;
@@ -623,17 +660,22 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             }
             uint8_t *slot = pring + s * kPSlot;
             if (part == 0) {
-              const uint32_t bytes = (int4_group ? (BM + BW) * 64u : kABytes) + BN * 4u +
+              const uint32_t bytes = (two_slots ? kABytes : (BM + BW) * 64u) + BN * 4u +
                                      (p.sa_by_tma ? BM * 4u : 0u);
               mbar_arrive_expect_tx(&pfull[s], bytes);
-              if (int4_group) {
+              if (!two_slots) {
                 tma_load_2d(slot, &maps.a4, wp.g * 64, arow, &pfull[s]);
                 tma_load_2d(slot + kPackWOff, &maps.w4, wp.g * 64, wrow, &pfull[s]);
               } else {
-                tma_load_2d(slot, &maps.a8, 0, arow, &pfull[s]);
+                // W4A4: the INT8 outlier tile of A ([M][128]); W4A8: group g of A ([M][K])
+                tma_load_2d(slot, &maps.a8, kA8 ? wp.g * 128 : 0, arow, &pfull[s]);
               }
               tma_load_2d(slot + kSwLinOff, &maps.sw, wp.n0, wp.g, &pfull[s]);
               if (p.sa_by_tma) tma_load_2d(slot + kSaLinOff, &maps.sa, arow, wp.g, &pfull[s]);
+            } else if (int4_group) {
+              // W4A8: the packed INT4 weight tile in the second slot
+              mbar_arrive_expect_tx(&pfull[s], BW * 64u);
+              tma_load_2d(slot, &maps.w4, wp.g * 64, wrow, &pfull[s]);
             } else {
               mbar_arrive_expect_tx(&pfull[s], kBBytes);
               tma_load_2d(slot, &maps.w8, 0, wrow, &pfull[s]);
@@ -700,6 +742,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
       for (int64_t it = 0; it < iters; ++it, ur.next(kNU), sr.next(kNS)) {
         const int u = ur.idx, sl = sr.idx;
         const bool int4_group = w.g < p.G - 1;
+        const bool two_slots = kA8 || !int4_group;
         const RingPos p0 = pr;
         RingPos p1 = pr;
         p1.next(kNP);
@@ -712,15 +755,17 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
           ok = mbar_wait(&uempty[u], ur.phase ^ 1u, abort_flag) &&
                mbar_wait(&sempty[sl], sr.phase ^ 1u, abort_flag) &&
                mbar_wait(&pfull[s0], p0.phase, abort_flag);
-        if (ok && !int4_group) ok = mbar_wait(&pfull[s1], p1.phase, abort_flag);
+        if (ok && two_slots) ok = mbar_wait(&pfull[s1], p1.phase, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) fail();
           break;
         }
         const uint8_t *pk = pring + s0 * kPSlot;
         uint8_t *op = uring + u * kUSlot;
-        if (int4_group)
+        if (!two_slots)
           unpack_int4(lt, pk, op);
+        else if (int4_group)
+          copy_a8_unpack_w4(lt, pk, pring + s1 * kPSlot, op);
         else
           copy_int8(lt, pk, pring + s1 * kPSlot, op);
         layout_scales(p, lt, pk, sring + sl * kSSlot, sa_d);
@@ -729,7 +774,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&pempty[s0]);
-          if (!int4_group) mbar_arrive(&pempty[s1]);
+          if (two_slots) mbar_arrive(&pempty[s1]);
           mbar_arrive(&sfull[sl]);
           if (rank == 0)
             mbar_arrive(&ufull[u]);
@@ -737,7 +782,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             mbar_arrive_remote(mfull_leader + 8u * u);
         }
         pr = p1;
-        if (!int4_group) pr.next(kNP);
+        if (two_slots) pr.next(kNP);
         w = wn;
       }
     }

@@ -78,18 +78,20 @@ __host__ __device__ inline QuantLayout quant_layout(int K, int stages_n) {
   return L;
 }
 
-// Gather rotation of lane `sub` (0..7) in team `team` (0..3) for a dense group.
-__device__ __forceinline__ int quant_rotation(int sub, int team) {
-  return 2 * ((sub >> 2) & 1) + 4 * team;
+// Gather rotation of lane `sub` (0..7) in team `team` (0..3) for a dense
+// group. With every group INT8 (a8) it is a whole number of 4-element words,
+// so that the 16 code bytes are put back in order by moving whole words.
+__device__ __forceinline__ int quant_rotation(int sub, int team, bool a8) {
+  return a8 ? 4 * team : 2 * ((sub >> 2) & 1) + 4 * team;
 }
 
 // Table slot of reordered position p: group g = p/128 is quantized by team
 // g%4 of some warp; lane sub = (p%128)/16 takes element e = p%16 at gather step
 // (e - rot) mod 16. Slots 0..7 of all 8 lanes come first, then slots 8..15, so
 // that each 8-lane team reads 128 contiguous bytes per 16-byte table load.
-__device__ __forceinline__ int quant_table_index(int p, int Gd) {
+__device__ __forceinline__ int quant_table_index(int p, int Gd, bool a8) {
   const int g = p >> 7, sub = (p >> 4) & 7, e = p & 15;
-  const int rot = g < Gd ? quant_rotation(sub, g & 3) : 0;
+  const int rot = (a8 || g < Gd) ? quant_rotation(sub, g & 3, a8) : 0;
   const int slot = (e - rot) & 15;
   return (((g * 2 + (slot >> 3)) * 8 + sub) << 3) + (slot & 7);
 }
@@ -99,7 +101,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
 reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t ld,
                      const int32_t *__restrict__ outlier_idx, uint8_t *__restrict__ q4,
                      int8_t *__restrict__ q8, float *__restrict__ scales, int stages_n,
-                     int crews_n) {
+                     int crews_n, int a8) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const QuantLayout L = quant_layout(K, stages_n * crews_n);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kQHdrFull);
@@ -206,13 +208,13 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
       const int b = __ffs(bits) - 1;
       bits &= bits - 1;
       if (pos < Kd)
-        table[quant_table_index(pos, Gd)] = static_cast<uint16_t>(2 * (w * 32 + 8 * qtr + b));
+        table[quant_table_index(pos, Gd, a8)] = static_cast<uint16_t>(2 * (w * 32 + 8 * qtr + b));
       ++pos;
     }
   }
   if (tid < 128) {
     const int c = oc;
-    if (c >= 0 && c < K) table[quant_table_index(Kd + tid, Gd)] = static_cast<uint16_t>(2 * c);
+    if (c >= 0 && c < K) table[quant_table_index(Kd + tid, Gd, a8)] = static_cast<uint16_t>(2 * c);
   }
   __syncthreads();
 
@@ -266,7 +268,9 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
   const int team = lane >> 3;
   const unsigned team_mask = 0xFFu << (8 * team);
   // Byte permutes that rotate the packed dense 8 bytes left by rot/2 bytes.
-  const int krot = quant_rotation(sub, team) >> 1;
+  const int krot = quant_rotation(sub, team, false) >> 1;
+  // INT8 groups: code words come out rotated by `wrot` words (a8 only)
+  const int wrot = a8 ? team : 0;
   uint32_t sel_lo = 0, sel_hi = 0;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -291,13 +295,13 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     const int64_t r = blockIdx.x + static_cast<int64_t>(i) * grid;
     const uint8_t *row = cstage + s * L.row_bytes;
     uint8_t *q4_r = q4 + r * q4_row;
-    int8_t *q8_r = q8 + r * 128;
+    int8_t *q8_r = q8 + r * (a8 ? static_cast<int64_t>(K) : 128);
     float *scales_r = scales + r;
 
     for (int gb = 0; gb < G; gb += 32) {
       const int g = gb + cw * 4 + team;
       if (g > Gd) continue;  // whole 8-lane teams skip together
-      const bool dense = g < Gd;
+      const bool dense = !a8 && g < Gd;
       const uint16_t *tb = table + ((g * 2) * 8 + sub) * 8;
       const uint4 oa = *reinterpret_cast<const uint4 *>(tb);       // slots 0..7
       const uint4 ob = *reinterpret_cast<const uint4 *>(tb + 64);  // slots 8..15
@@ -339,12 +343,18 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
         *reinterpret_cast<uint2 *>(q4_r + g * 64 + sub * 8) =
             make_uint2(__byte_perm(lo, hi, sel_lo), __byte_perm(lo, hi, sel_hi));
       } else {
+        // gather slot e holds element (e + 4*wrot) mod 16: word j of the
+        // output is slot word (j - wrot) mod 4
+        const uint32_t w0 = low_bytes4(b[0], b[1], b[2], b[3]);
+        const uint32_t w1 = low_bytes4(b[4], b[5], b[6], b[7]);
+        const uint32_t w2 = low_bytes4(b[8], b[9], b[10], b[11]);
+        const uint32_t w3 = low_bytes4(b[12], b[13], b[14], b[15]);
         uint4 o;
-        o.x = low_bytes4(b[0], b[1], b[2], b[3]);
-        o.y = low_bytes4(b[4], b[5], b[6], b[7]);
-        o.z = low_bytes4(b[8], b[9], b[10], b[11]);
-        o.w = low_bytes4(b[12], b[13], b[14], b[15]);
-        *reinterpret_cast<uint4 *>(q8_r + sub * 16) = o;
+        o.x = wrot == 0 ? w0 : wrot == 1 ? w3 : wrot == 2 ? w2 : w1;
+        o.y = wrot == 0 ? w1 : wrot == 1 ? w0 : wrot == 2 ? w3 : w2;
+        o.z = wrot == 0 ? w2 : wrot == 1 ? w1 : wrot == 2 ? w0 : w3;
+        o.w = wrot == 0 ? w3 : wrot == 1 ? w2 : wrot == 2 ? w1 : w0;
+        *reinterpret_cast<uint4 *>(q8_r + (a8 ? g * 128 : 0) + sub * 16) = o;
       }
       if (sub == 0) scales_r[static_cast<int64_t>(g) * rows] = scale;
     }
