@@ -162,3 +162,40 @@ def test_header_compiles_as_plain_c(tmp_path):
     r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-I",
                         os.path.join(ROOT, "include"), str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def gemm_quant(lib, M=16, N=256, K=512, n_out=128, group=128, qy4=A16, qy8=A16, sy=A16, qa4=A16):
+    return lib.atom_w4a4_gemm_quant(qa4, A16, A16, A16, A16, A16, M, N, K, n_out, group,
+                                    qy4, qy8, sy, None)
+
+
+def test_quantizing_gemm_checks_arguments_on_the_host(lib):
+    assert gemm_quant(lib, M=0) == OK
+    assert gemm_quant(lib, N=200) == SHAPE            # not whole 128-column groups
+    assert gemm_quant(lib, N=128) == SHAPE            # needs an INT4 group and the INT8 group
+    assert gemm_quant(lib, N=32768 + 128) == SHAPE    # above the next layer's largest K
+    assert gemm_quant(lib, qy4=0) == INVALID
+    assert gemm_quant(lib, sy=0) == INVALID
+    assert gemm_quant(lib, qy8=A16 + 8) == ALIGN
+    assert gemm_quant(lib, sy=MIS) == ALIGN
+    assert gemm_quant(lib, qa4=MIS) == ALIGN
+    assert gemm_quant(lib, group=64) == UNSUPPORTED
+
+
+def test_w4a8_entry_points_check_arguments_on_the_host(lib):
+    q = lib.atom_reorder_quant_a8
+    assert q(A16, 0, 512, 512, A16, 128, 128, A16, A16, None) == OK
+    assert q(A16, 4, 500, 504, A16, 128, 128, A16, A16, None) == SHAPE
+    assert q(A16, 4, 512, 512, A16, 128, 128, 0, A16, None) == INVALID
+    assert q(A16, 4, 512, 512, A16, 128, 128, A16 + 8, A16, None) == ALIGN
+    assert q(A16, 4, 512, 512, A16, 128, 64, A16, A16, None) == UNSUPPORTED
+    g = lib.atom_w4a8_gemm
+    args = [A16] * 5
+    assert g(*args, A16, 0, 256, 512, 128, 128, None) == OK
+    assert g(*args, 0, 16, 256, 512, 128, 128, None) == INVALID       # no y
+    assert g(*args, A16, 16, 260, 512, 128, 128, None) == SHAPE       # N % 8 != 0
+    assert g(MIS, *args[1:], A16, 16, 256, 512, 128, 128, None) == ALIGN
+    assert g(*args, A16, 16, 256, 512, 64, 128, None) == UNSUPPORTED
+    p = lib.atom_w4a8_gemm_partials
+    assert p(*args, 0, A16, 16, 256, 512, 128, 128, None) == INVALID  # no partials buffer
+    assert p(*args, A16 + 4, None, 16, 256, 512, 128, 128, None) == ALIGN
