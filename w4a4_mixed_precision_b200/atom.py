@@ -117,6 +117,38 @@ def _dev(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
     return t.data_ptr()
 
 
+MAX_K = 32768   # the largest K the library accepts (include/atom.h)
+
+
+def _valid_k(K: int) -> bool:
+    return K % GROUP == 0 and 2 * GROUP <= K <= MAX_K
+
+
+def _expect_shape(t: torch.Tensor, shape, name: str) -> None:
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _check_quantized(q, K: int, name: str, rows: Optional[int] = None) -> None:
+    """Shapes of a quantized operand (Quantized) for K. Only checked for a K the
+    library accepts: it reports any other K itself, with its own status."""
+    if not _valid_k(K):
+        return
+    rows = q.q4.shape[0] if rows is None else rows
+    _expect_shape(q.q4, (rows, (K - N_OUTLIER) // 2), name + ".q4")
+    _expect_shape(q.q8, (rows, N_OUTLIER), name + ".q8")
+    _expect_shape(q.scales, (K // GROUP, rows), name + ".scales")
+
+
+def _check_quantized_a8(q, K: int, name: str, rows: Optional[int] = None) -> None:
+    """Shapes of W4A8 activations (QuantizedA8) for K, as _check_quantized."""
+    if not _valid_k(K):
+        return
+    rows = q.q8.shape[0] if rows is None else rows
+    _expect_shape(q.q8, (rows, K), name + ".q8")
+    _expect_shape(q.scales, (K // GROUP, rows), name + ".scales")
+
+
 class Quantized(NamedTuple):
     """One quantized operand: INT4 codes, INT8 outlier codes, group-major scales."""
     q4: torch.Tensor
@@ -142,6 +174,7 @@ def _quant(fn: str, x: torch.Tensor, outlier_idx: torch.Tensor, out: Optional[Qu
         raise ValueError("input rows must be contiguous")
     if out is None:
         out = empty_quantized(rows, K, x.device)
+    _check_quantized(out, K, "out", rows)
     if not x.is_cuda or x.dtype != torch.float16:
         raise ValueError("input must be a CUDA float16 tensor")
     st = getattr(lib(), fn)(x.data_ptr(), rows, K, x.stride(0),
@@ -177,6 +210,7 @@ def atom_reorder_quant_a8(x: torch.Tensor, outlier_idx: torch.Tensor,
     if out is None:
         out = QuantizedA8(torch.empty((rows, K), dtype=torch.int8, device=x.device),
                           torch.empty((K // GROUP, rows), dtype=torch.float32, device=x.device))
+    _check_quantized_a8(out, K, "out", rows)
     st = lib().atom_reorder_quant_a8(x.data_ptr(), rows, K, x.stride(0),
                                      _dev(outlier_idx, torch.int32, "outlier_idx"),
                                      outlier_idx.numel(), GROUP, _dev(out.q8, torch.int8, "q8"),
@@ -189,8 +223,11 @@ def atom_w4a8_gemm(qa: QuantizedA8, qw: Quantized, K: int, y: Optional[torch.Ten
                    stream=None) -> torch.Tensor:
     """W4A8: Y fp16 [M, N] from INT8 activations and the W4A4 weights (see include/atom.h)."""
     M, N = qa.rows, qw.rows
+    _check_quantized_a8(qa, K, "qa")
+    _check_quantized(qw, K, "qw")
     if y is None:
         y = torch.empty((M, N), dtype=torch.float16, device=qa.q8.device)
+    _expect_shape(y, (M, N), "y")
     st = lib().atom_w4a8_gemm(
         _dev(qa.q8, torch.int8, "qa8"), _dev(qa.scales, torch.float32, "sa"),
         _dev(qw.q4, torch.uint8, "qw4"), _dev(qw.q8, torch.int8, "qw8"),
@@ -204,6 +241,8 @@ def atom_w4a8_gemm_partials(qa: QuantizedA8, qw: Quantized, K: int, stream=None)
     """Debug entry of the W4A8 GEMM: per-group int32 partial sums [G, M, N] and Y."""
     M, N = qa.rows, qw.rows
     dev = qa.q8.device
+    _check_quantized_a8(qa, K, "qa")
+    _check_quantized(qw, K, "qw")
     partials = torch.empty((K // GROUP, M, N), dtype=torch.int32, device=dev)
     y = torch.empty((M, N), dtype=torch.float16, device=dev)
     st = lib().atom_w4a8_gemm_partials(
@@ -237,8 +276,11 @@ def atom_w4a4_gemm(qa: Quantized, qw: Quantized, K: int, y: Optional[torch.Tenso
     allocated here. `split=False` runs without a workspace (no K split)."""
     M, N = qa.rows, qw.rows
     dev = qa.q4.device
+    _check_quantized(qa, K, "qa")
+    _check_quantized(qw, K, "qw")
     if y is None:
         y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    _expect_shape(y, (M, N), "y")
     if workspace is None and split:
         workspace = gemm_workspace(M, N, K, dev)
     ws_ptr, ws_bytes = (None, 0) if workspace is None or not split else (
@@ -258,8 +300,11 @@ def atom_w4a4_gemm_noalloc(qa: Quantized, qw: Quantized, K: int,
     of K keeps its partials in the library's fixed 8 MiB device array (see
     include/atom.h). Pass `y` to keep this wrapper allocation-free as well."""
     M, N = qa.rows, qw.rows
+    _check_quantized(qa, K, "qa")
+    _check_quantized(qw, K, "qw")
     if y is None:
         y = torch.empty((M, N), dtype=torch.float16, device=qa.q4.device)
+    _expect_shape(y, (M, N), "y")
     st = lib().atom_w4a4_gemm_noalloc(
         _dev(qa.q4, torch.uint8, "qa4"), _dev(qa.q8, torch.int8, "qa8"),
         _dev(qa.scales, torch.float32, "sa"), _dev(qw.q4, torch.uint8, "qw4"),
@@ -276,10 +321,16 @@ def atom_w4a4_gemm_partials(qa: Quantized, qw: Quantized, K: int,
     """Debug entry: per-group int32 partial sums [G, M, N] (and Y unless want_y is False)."""
     M, N = qa.rows, qw.rows
     dev = qa.q4.device
+    _check_quantized(qa, K, "qa")
+    _check_quantized(qw, K, "qw")
     if partials is None:
         partials = torch.empty((K // GROUP, M, N), dtype=torch.int32, device=dev)
+    if _valid_k(K):
+        _expect_shape(partials, (K // GROUP, M, N), "partials")
     if want_y and y is None:
         y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    if want_y:
+        _expect_shape(y, (M, N), "y")
     st = lib().atom_w4a4_gemm_partials(
         _dev(qa.q4, torch.uint8, "qa4"), _dev(qa.q8, torch.int8, "qa8"),
         _dev(qa.scales, torch.float32, "sa"), _dev(qw.q4, torch.uint8, "qw4"),
@@ -297,8 +348,11 @@ def atom_w4a4_gemm_quant(qa: Quantized, qw: Quantized, K: int, out: Optional[Qua
     and scales atom_reorder_quant would write for Y (unsplit, fp16) with Y's last 128
     columns as the outlier channels (see include/atom.h). N must be a multiple of 128."""
     M, N = qa.rows, qw.rows
+    _check_quantized(qa, K, "qa")
+    _check_quantized(qw, K, "qw")
     if out is None:
         out = empty_quantized(M, N, qa.q4.device)
+    _check_quantized(out, N, "out", M)   # Y's N is the next layer's K
     st = lib().atom_w4a4_gemm_quant(
         _dev(qa.q4, torch.uint8, "qa4"), _dev(qa.q8, torch.int8, "qa8"),
         _dev(qa.scales, torch.float32, "sa"), _dev(qw.q4, torch.uint8, "qw4"),
