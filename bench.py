@@ -178,6 +178,133 @@ def cpu_oracle_run(w, A, W, idx, budget_s: float, min_rows: int = 8):
     return 2.0 * rows * w.N * w.K / dt, rows, dt, cores
 
 
+# ----------------------------------------------------------------------------- per-config legs
+
+
+def _time_cycle(fns, n, stream):
+    """Average ms per call of `fns` called round-robin n times back to back on
+    `stream` (three untimed calls first), timed with CUDA events on that stream."""
+    import torch
+    for i in range(3):
+        fns[i % len(fns)]()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        fns[i % len(fns)]()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def _copies_for(bytes_per_set: float, cap: int = 16) -> int:
+    """Input sets to rotate through so that consecutive calls never find their
+    operands in the 126 MB L2 (at least two sets, and more than twice L2)."""
+    return int(min(cap, max(2, -(-2 * L2_BYTES // max(bytes_per_set, 1)))))
+
+
+def int8_probe_tops(stream, groups: int = 4096, reps: int = 5):
+    """Dense INT8 tensor-core rate measured by the library's probe loop
+    (atom_probe_mma_i8: the GEMM's 2-SM MMA shape back to back, no data
+    movement); the median of `reps` timed launches after two untimed ones."""
+    import torch
+    from w4a4_mixed_precision_b200 import atom
+    ops = 0
+    for _ in range(2):
+        ops = atom.atom_probe_mma_i8(groups, stream=stream)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        atom.atom_probe_mma_i8(groups, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    if atom.atom_device_status(clear=True) != 0:
+        raise RuntimeError("device status set by the INT8 probe")
+    return ops / (ms * 1e-3) / 1e12, ms
+
+
+def per_config_legs(configs, dev, stream, n_calls, int8_peak, int8_probe, hbm_gbs):
+    """Throughput of the other Llama-shaped workloads, each on its own seeded
+    inputs, with input sets rotated so that no call finds its operands in L2:
+    the decode GEMM (latency and GB/s of its algorithmic bytes against HBM), the
+    prefill and down-projection GEMMs (TOPS against the int8 denominators), the
+    quantizer (GB/s against HBM), and fp16 cuBLAS of the same shape beside each."""
+    import torch
+    from w4a4_mixed_precision_b200 import atom, inputs
+    out = {}
+    for c in configs:
+        w = inputs.workload(c)
+        Kd, G = w.K - 128, w.K // 128
+        A_h, W_h, idx_h = inputs.activations(c), inputs.weights(c), inputs.outlier_channels(c)
+        A = torch.from_numpy(A_h.view(np.uint16)).to(dev).view(torch.float16)
+        W16 = torch.from_numpy(W_h.view(np.uint16)).to(dev).view(torch.float16)
+        idx = torch.from_numpy(idx_h).to(dev)
+        del A_h, W_h
+        qw0 = atom.atom_quant_weights(W16, idx)
+        qa0 = atom.atom_reorder_quant(A, idx)
+        packed_row = Kd // 2 + 128 + 4 * G
+        gemm_bytes = (w.M + w.N) * packed_row + w.M * w.N * 2
+        quant_bytes = w.M * (2 * w.K + packed_row)
+        ops = 2.0 * w.M * w.N * w.K
+        n_sets = _copies_for(gemm_bytes)
+        qas = [qa0] + [atom.Quantized(*(t.clone() for t in qa0)) for _ in range(n_sets - 1)]
+        qws = [qw0] + [atom.Quantized(*(t.clone() for t in qw0)) for _ in range(n_sets - 1)]
+        ys = [torch.empty((w.M, w.N), dtype=torch.float16, device=dev) for _ in range(n_sets)]
+        wss = [atom.gemm_workspace(w.M, w.N, w.K, dev) for _ in range(n_sets)]
+
+        def gemm_fn(i):
+            return lambda: atom.atom_w4a4_gemm(qas[i], qws[i], w.K, y=ys[i], stream=stream,
+                                               workspace=wss[i])
+        g_ms = _time_cycle([gemm_fn(i) for i in range(n_sets)], n_calls, stream)
+        n_qsets = _copies_for(quant_bytes)
+        As = [A] + [A.clone() for _ in range(n_qsets - 1)]
+        qouts = [atom.empty_quantized(w.M, w.K, dev) for _ in range(n_qsets)]
+
+        def quant_fn(i):
+            return lambda: atom.atom_reorder_quant(As[i], idx, out=qouts[i], stream=stream)
+        q_ms = _time_cycle([quant_fn(i) for i in range(n_qsets)], n_calls, stream)
+        del As, qouts, qas, ys, wss
+        n_csets = _copies_for(2.0 * (w.M + w.N) * w.K + 2.0 * w.M * w.N)
+        Ws = [W16] + [W16.clone() for _ in range(n_csets - 1)]
+        yc = torch.empty((w.M, w.N), dtype=torch.float16, device=dev)
+        c_ms = _time_cycle([(lambda Wi: (lambda: torch.matmul(A, Wi.t(), out=yc)))(Wi)
+                            for Wi in Ws], n_calls, stream)
+        del Ws, yc, W16, A
+        if atom.atom_device_status(clear=True) != 0:
+            raise RuntimeError(f"device status set on workload {c}")
+        g_tops = ops / (g_ms * 1e-3) / 1e12
+        entry = {
+            "workload": f"{w.name} M={w.M} N={w.N} K={w.K}",
+            "gemm_us": round(g_ms * 1e3, 2),
+            "gemm_tops": round(g_tops, 2),
+            "gemm_frac_int8_peak": round(g_tops / int8_peak, 4),
+            "gemm_frac_int8_probe": round(g_tops / int8_probe, 4) if int8_probe else None,
+            "gemm_algorithmic_bytes": gemm_bytes,
+            "gemm_gbs": round(gemm_bytes / (g_ms * 1e-3) / 1e9, 1),
+            "gemm_frac_hbm": round(gemm_bytes / (g_ms * 1e-3) / 1e9 / hbm_gbs, 4),
+            "gemm_splits_workspace_bytes": atom.atom_gemm_workspace_bytes(w.M, w.N, w.K),
+            "quant_us": round(q_ms * 1e3, 2),
+            "quant_bytes": quant_bytes,
+            "quant_gbs": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
+            "quant_frac_hbm": round(quant_bytes / (q_ms * 1e-3) / 1e9 / hbm_gbs, 4),
+            "fp16_cublas_us": round(c_ms * 1e3, 2),
+            "fp16_cublas_tflops": round(ops / (c_ms * 1e-3) / 1e12, 2),
+            "w4a4_gemm_speedup_vs_fp16": round(c_ms / g_ms, 3),
+            "calls": n_calls,
+            "l2": f"GEMM rotates {n_sets} input sets, quantizer {n_qsets}, cuBLAS {n_csets} "
+                  f"weight copies (each rotation more than twice the 126 MB L2, or 16 sets)",
+            "bound": "hbm" if c == 1 else "tensor",
+        }
+        out[w.name] = entry
+    return out
+
+
 # ----------------------------------------------------------------------------- main
 
 
@@ -204,6 +331,10 @@ def main():
                     help="skip the INT4 KV-cache quantize/dequantize measurement")
     ap.add_argument("--m", type=int, default=None,
                     help="use only the first M activation rows (small profiling cases)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the decode / prefill / down-projection workloads (1, 2, 3)")
+    ap.add_argument("--no-probe", action="store_true",
+                    help="skip the INT8 tensor-core peak probe (second GEMM denominator)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -307,7 +438,7 @@ def main():
         ev_quant = [torch.cuda.Event() for _ in range(2)]
         ev_gemm = [torch.cuda.Event() for _ in range(2)]
         ev_d2h = [torch.cuda.Event() for _ in range(2)]
-        e2e_steps = max(3, min(20, n_steps // 10))
+        e2e_steps = max(10, min(20, n_steps // 2))
 
         def e2e_step(i):
             b = i % 2
@@ -420,6 +551,24 @@ def main():
         if atom.atom_device_status(clear=True) != 0:
             raise RuntimeError("device status set by the W4A8 variant")
 
+    # -------- the dense INT8 tensor-core rate (second denominator) and the other workloads
+    peaks, peak_kind = _peaks()
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    probe = None
+    if not args.no_probe:
+        probe_tops, probe_ms = int8_probe_tops(stream)
+        probe = {"value": round(probe_tops, 1), "unit": "TOPS", "ms": round(probe_ms, 4),
+                 "kind": "atom_probe_mma_i8: tcgen05.mma.cta_group::2.kind::i8 M=256 N=256 "
+                         "K=32 back to back on every CTA pair (one CTA per SM), zero operands "
+                         "in shared memory, no loads or dequantization; median of 5 launches"}
+    per_config = None
+    if not args.no_per_config and args.m is None and args.workload == WORKLOAD_INDEX:
+        with ClockSampler(torch.cuda.current_device()) as pc_clocks:
+            per_config = per_config_legs((1, 2, 3), dev, stream, max(10, min(50, n_steps)),
+                                         int8_peak, probe["value"] if probe else None,
+                                         peaks["hbm_gbs"])
+        per_config["clocks"] = pc_clocks.summary()
+
     # -------- fp16 cuBLAS GEMM of the same shape (torch.matmul), a library baseline
     cublas = None
     if not args.no_cublas:
@@ -528,13 +677,11 @@ def main():
     if rank != 0:
         return
 
-    peaks, peak_kind = _peaks()
     ops = 2.0 * w.M * w.N * w.K
     ms_per_step = elapsed_ms / n_steps
     value = ops * world / (ms_per_step * 1e-3) / 1e12
     gemm_avg = statistics.mean(gemm_ms)
     quant_avg = statistics.mean(quant_ms)
-    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
     gemm_tops = ops / (gemm_avg * 1e-3) / 1e12
     Kd = w.K - 128
     quant_bytes = w.M * (2 * w.K + Kd // 2 + 128 + 4 * (w.K // 128))
@@ -559,6 +706,7 @@ def main():
         "config": workload_cfg,
         "gemm_tops": round(gemm_tops, 2),
         "gemm_frac_int8_peak": round(gemm_tops / int8_peak, 4),
+        "gemm_frac_int8_probe": round(gemm_tops / probe["value"], 4) if probe else None,
         "quant_gbs": round(quant_gbs, 1),
         "quant_frac_hbm": round(quant_gbs / peaks["hbm_gbs"], 4),
         "kernel_ms": {"reorder_quant": round(quant_avg, 4), "w4a4_gemm": round(gemm_avg, 4)},
@@ -573,6 +721,7 @@ def main():
             "algorithmic_bytes": gemm_bytes,
             "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
                            f"{INT8_OVER_BF16} (nominal int8:bf16 ratio)",
+            "frac_of_int8_probe": round(gemm_tops / probe["value"], 4) if probe else None,
         },
         "roofline_quant": {
             "kernel": "reorder_quant_kernel",
@@ -589,6 +738,10 @@ def main():
         "gpu_launches": 2 * n_steps,
         "e2e": e2e,
     }
+    if probe is not None:
+        line["int8_probe"] = probe
+    if per_config is not None:
+        line["per_config"] = per_config
     if cublas is not None:
         cublas["w4a4_gemm_speedup"] = round(cublas["ms"] / gemm_avg, 3)
         line["fp16_cublas"] = cublas

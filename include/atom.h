@@ -33,8 +33,17 @@
  *    atom_device_status() reads.
  *  - Inputs must be finite.
  *
- * Thread safety: the entry points keep no host state except a per-device
- * cache of the SM count; concurrent calls on different streams are safe.
+ * Thread safety: the host side keeps one per-device cache of launch facts
+ * (SM count, shared-memory limits, co-resident CTA pairs), filled once under a
+ * lock; calls from several host threads are safe. Two kinds of device state are
+ * shared by every call on a device, whatever its stream:
+ *  - the device status word (see atom_device_status): an error recorded by a
+ *    kernel on one stream is what the next atom_device_status() reports, even
+ *    if the caller is checking a different stream's work;
+ *  - the fixed scratch array of atom_w4a4_gemm_noalloc: calls of that entry
+ *    point that overlap on the GPU race on it and must be ordered by the caller.
+ * Apart from these, calls on different streams that share no output buffer and
+ * no workspace may run concurrently.
  */
 #ifndef ATOM_B200_H
 #define ATOM_B200_H
@@ -249,24 +258,26 @@ ATOM_API size_t atom_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
  * atom_w4a4_gemm_noalloc -- atom_w4a4_gemm for callers that cannot allocate
- * device memory around the call: code running while a CUDA graph is captured,
- * serving runtimes that give all device memory to a fixed pool at start-up, C
- * callers with no device allocator. (The pages describe no such entry point;
- * it is a deployment convenience of this library.)
+ * device memory around the call: serving runtimes that hand all device memory
+ * to a fixed pool at start-up (there is nothing left to allocate from), and C
+ * or embedded callers that have no device allocator of their own. (The pages
+ * have no counterpart; it is a deployment convenience of this library.)
  *
  * Arguments, layouts, result and errors are those of atom_w4a4_gemm without
- * the workspace. When the shape splits K (small M), the split's fp32 partial
- * tiles go to a fixed 8 MiB array in the library's device memory instead of a
- * caller workspace; every GPU that loads the library holds that array until
- * the process exits. A shape whose partials would need more than 8 MiB
- * (splits * M * N * 4 bytes, see atom_gemm_workspace_bytes) returns
- * ATOM_ERR_SHAPE before anything is launched. The call allocates nothing.
+ * the workspace. When the shape splits K through a workspace (M > 64 with few
+ * output tiles), the split's fp32 partial tiles go to a fixed 8 MiB array in
+ * the library's device memory instead of a caller workspace; every GPU that
+ * loads the library holds that array until the process exits. A shape whose
+ * partials would need more than 8 MiB (the value atom_gemm_workspace_bytes
+ * reports) returns ATOM_ERR_SHAPE before anything is launched. The call
+ * allocates nothing.
  *
  * All calls on a device share the array, and a call leaves its partials in
  * it: two calls that overlap on the GPU (other streams, other host threads)
  * race and must be ordered by the caller. The first call on each device does
- * a one-time set-up (it looks up the array's device address and the kernel's
- * launch limits) and should come before any stream capture.
+ * a one-time set-up with that device current (it looks up the array's device
+ * address with cudaGetSymbolAddress and the kernel's launch limits); make that
+ * first call before any stream capture.
  */
 ATOM_API atom_status_t atom_w4a4_gemm_noalloc(const uint8_t *qa4, const int8_t *qa8,
                                               const float *sa, const uint8_t *qw4,
@@ -329,6 +340,40 @@ ATOM_API atom_status_t atom_kv_quant(const void *x, int64_t groups, uint8_t *q4,
                                      atom_stream_t stream);
 ATOM_API atom_status_t atom_kv_dequant(const uint8_t *q4, const float *scales, int64_t groups,
                                        void *out, atom_stream_t stream);
+
+/*
+ * atom_probe_mma_i8 -- a measurement aid (the pages have no counterpart): the
+ * dense INT8 tensor-core rate of this GPU, the second roofline denominator of
+ * the W4A4 GEMM. Every CTA pair the GPU holds at once (one CTA per SM) issues
+ * `groups` groups of four tcgen05.mma.cta_group::2.kind::i8 of the GEMM's shape
+ * (M = 256, N = 256, K = 32, zero-filled operands in shared memory) into two
+ * alternating TMEM accumulators, with no loads and no dequantization. The
+ * launch performs 2 * 256 * 256 * 128 * groups * (*pairs_out) integer
+ * operations; the caller times it on `stream`.
+ *
+ *   groups     1 <= groups <= 2^20 (else ATOM_ERR_INVALID_ARG).
+ *   pairs_out  host int32 (output): the number of CTA pairs launched.
+ * Stream-ordered, allocates nothing.
+ */
+ATOM_API atom_status_t atom_probe_mma_i8(int64_t groups, int32_t *pairs_out,
+                                         atom_stream_t stream);
+
+/*
+ * atom_debug_wait_timeout -- a test aid for the library's failure detection
+ * (the pages have no counterpart). Every pipeline wait in the GEMM and
+ * quantizer kernels is bounded: a wait that runs past its limit gives up,
+ * records ATOM_ERR_TIMEOUT in the device status word and lets the kernel end,
+ * instead of hanging the GPU. This entry point runs that same bounded wait
+ * (the same device function) in a one-thread kernel on an mbarrier that
+ * nothing ever arrives on and that no copy or MMA is tied to, with a limit of
+ * `limit_ns` nanoseconds in place of the production 1 s. The kernel therefore
+ * gives up after about `limit_ns`, and the next atom_device_status() reports
+ * ATOM_ERR_TIMEOUT. Nothing is left in flight; the context stays usable.
+ *
+ *   limit_ns  0 < limit_ns <= 1e9 (else ATOM_ERR_INVALID_ARG).
+ * Stream-ordered, allocates nothing.
+ */
+ATOM_API atom_status_t atom_debug_wait_timeout(uint64_t limit_ns, atom_stream_t stream);
 
 /*
  * atom_device_status -- first device-detected error since the last clear on the

@@ -199,3 +199,10 @@ def test_w4a8_entry_points_check_arguments_on_the_host(lib):
     p = lib.atom_w4a8_gemm_partials
     assert p(*args, 0, A16, 16, 256, 512, 128, 128, None) == INVALID  # no partials buffer
     assert p(*args, A16 + 4, None, 16, 256, 512, 128, 128, None) == ALIGN
+
+
+def test_timeout_aid_validates_its_limit_on_the_host(lib):
+    """atom_debug_wait_timeout rejects a zero limit and one above the
+    production 1 s before touching the device."""
+    assert lib.atom_debug_wait_timeout(0, None) == INVALID
+    assert lib.atom_debug_wait_timeout(2_000_000_000, None) == INVALID

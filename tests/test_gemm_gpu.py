@@ -1,10 +1,11 @@
 """Parity of the tcgen05 W4A4 GEMM with the CPU oracle.
 
 Per-group int32 partial sums must be bit-identical (debug entry point, full
-tensor on small shapes, 256x256 windows of the large workloads); the fp16
-output must be within the tolerance of gpu_util.y_rel_err of the oracle's
-fp64 output, on every row for small shapes and on seeded sampled rows for the
-full-size workloads (run exactly as the benchmark launches them)."""
+tensor on small shapes and on the decode workload, 256x256 windows of the large
+workloads; M <= 64 goes through the small-M kernel, as in production); the
+fp16 output must be within the tolerance of gpu_util.y_rel_err of the oracle's
+fp64 output, on every row of small shapes and of workloads 1 and 2, and on 512
+seeded rows of workloads 3 and 4 (run exactly as the benchmark launches them)."""
 import numpy as np
 import pytest
 import torch
@@ -97,6 +98,44 @@ def test_lossless_integers_give_the_exact_integer_matmul(c_oracle):
     assert np.array_equal(y, ref.astype(np.float64))
 
 
+@pytest.mark.parametrize("M,N,K,seed", [(1, 264, 1024, 51), (16, 4096, 4096, 52),
+                                        (40, 520, 2048, 53), (64, 392, 32768, 54),
+                                        (33, 128, 256, 55)])
+def test_small_m_kernel_partials_bit_exact(c_oracle, M, N, K, seed):
+    """M <= 64 runs the small-M kernel (weights on the MMA's M side) for the
+    partials entry point as for atom_w4a4_gemm: its per-group int32 partials
+    must equal the oracle's, and its unsplit Y must equal atom_w4a4_gemm's
+    unsplit Y bit for bit (same kernel, same order)."""
+    A, W, idx = inputs.random_case(seed, M, N, K, dist="t", param=3.0, outlier_factor=50.0,
+                                   sorted_outliers=(seed % 2 == 0))
+    P_ref, Y64 = _oracle_all(c_oracle, A, W, idx)
+    qa, qw = quant_dev(A, idx), quant_dev(W, idx, weights=True)
+    P, y = atom.atom_w4a4_gemm_partials(qa, qw, K)
+    y_plain = atom.atom_w4a4_gemm(qa, qw, K, split=False)
+    torch.cuda.synchronize()
+    P = P.cpu().numpy()
+    mism = np.argwhere(P != P_ref)
+    assert mism.size == 0, f"{len(mism)} partial mismatches, first {mism[:3].tolist()}"
+    y = y.cpu().numpy()
+    assert y_rel_err(y, Y64) <= Y_TOL
+    assert np.array_equal(y.view(np.uint16), y_plain.cpu().numpy().view(np.uint16))
+
+
+def test_decode_workload_partials_bit_exact_in_full(c_oracle):
+    """Every per-group partial of the full 64 x 4096 x 4096 decode workload,
+    computed by the small-M kernel, equals the oracle's."""
+    c = 1
+    w = inputs.workload(c)
+    A, W, idx = inputs.activations(c), inputs.weights(c), inputs.outlier_channels(c)
+    qa, qw = quant_dev(A, idx), quant_dev(W, idx, weights=True)
+    P, _ = atom.atom_w4a4_gemm_partials(qa, qw, w.K, want_y=False)
+    P = P.cpu().numpy()
+    ra, rw = c_oracle.quantize(A, idx), c_oracle.quantize(W, idx)
+    P_ref = c_oracle.partials(ra[0], ra[1], rw[0], rw[1], w.K)
+    mism = np.argwhere(P != P_ref)
+    assert mism.size == 0, f"{len(mism)} partial mismatches, first {mism[:3].tolist()}"
+
+
 @pytest.mark.parametrize("c", [1, 2, 3, 4])
 def test_partials_window_bit_exact_full_size_workload(c_oracle, c):
     """A 256x256 window of the per-group partials of a full-size workload."""
@@ -118,19 +157,29 @@ def test_partials_window_bit_exact_full_size_workload(c_oracle, c):
     assert np.array_equal(P, P_ref)
 
 
+# Rows of full-size Y compared with the oracle: every row of workloads 1 and 2,
+# and 512 seeded rows (always including the last) of workloads 3 and 4.
+FULL_Y_ROWS = {1: None, 2: None, 3: 512, 4: 512}
+
+
 @pytest.mark.parametrize("c", [1, 2, 3, 4])
-def test_full_size_output_on_sampled_rows(c_oracle, c):
-    """The full-size GEMM exactly as the benchmark launches it; Y checked on
-    seeded sampled rows (all N columns) against the oracle's fp64 output."""
+def test_full_size_output(c_oracle, c):
+    """The full-size GEMM exactly as the benchmark launches it; Y checked on all
+    N columns of every row (workloads 1, 2) or of 512 seeded rows (3, 4)
+    against the oracle's fp64 output."""
     w = inputs.workload(c)
     A, W, idx = inputs.activations(c), inputs.weights(c), inputs.outlier_channels(c)
     qa, qw = quant_dev(A, idx), quant_dev(W, idx, weights=True)
     y = atom.atom_w4a4_gemm(qa, qw, w.K)
     torch.cuda.synchronize()
-    rng = np.random.default_rng(200 + c)
-    n_rows = min(w.M, 32)
-    rows = np.sort(rng.choice(w.M, n_rows, replace=False))
-    rows[-1] = w.M - 1                                      # always include the last row
+    n_rows = FULL_Y_ROWS[c]
+    if n_rows is None or n_rows >= w.M:
+        rows = np.arange(w.M)
+    else:
+        rng = np.random.default_rng(200 + c)
+        rows = np.sort(rng.choice(w.M - 1, n_rows - 1, replace=False))
+        rows = np.append(rows, w.M - 1)                     # always include the last row
+    assert len(np.unique(rows)) == len(rows) == min(w.M, n_rows or w.M)
     ys = y[torch.from_numpy(rows).cuda()].cpu().numpy()
     ra = c_oracle.quantize(np.ascontiguousarray(A[rows]), idx)
     rw = c_oracle.quantize(W, idx)

@@ -66,6 +66,8 @@ SIGNATURES = {
     "atom_kv_quant": ([ct.c_void_p, ct.c_int64, ct.c_void_p, ct.c_void_p, ct.c_void_p], ct.c_int),
     "atom_kv_dequant": ([ct.c_void_p, ct.c_void_p, ct.c_int64, ct.c_void_p, ct.c_void_p],
                         ct.c_int),
+    "atom_debug_wait_timeout": ([ct.c_uint64, ct.c_void_p], ct.c_int),
+    "atom_probe_mma_i8": ([ct.c_int64, ct.POINTER(ct.c_int32), ct.c_void_p], ct.c_int),
     "atom_device_status": ([ct.c_int], ct.c_int),
     "atom_status_string": ([ct.c_int], ct.c_char_p),
     "atom_version": ([], ct.c_int),
@@ -296,9 +298,11 @@ def atom_w4a4_gemm(qa: Quantized, qw: Quantized, K: int, y: Optional[torch.Tenso
 
 def atom_w4a4_gemm_noalloc(qa: Quantized, qw: Quantized, K: int,
                            y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """atom_w4a4_gemm for callers that cannot allocate around the call: a split
-    of K keeps its partials in the library's fixed 8 MiB device array (see
-    include/atom.h). Pass `y` to keep this wrapper allocation-free as well."""
+    """atom_w4a4_gemm for callers that cannot allocate device memory around the
+    call (a runtime whose device memory all sits in a fixed pool, a C caller
+    without an allocator): a split of K keeps its partials in the library's
+    fixed 8 MiB device array (see include/atom.h). Pass `y` to keep this wrapper
+    allocation-free as well."""
     M, N = qa.rows, qw.rows
     _check_quantized(qa, K, "qa")
     _check_quantized(qw, K, "qw")
@@ -415,6 +419,21 @@ def atom_kv_dequant(q4: torch.Tensor, scales: torch.Tensor, out: Optional[torch.
 
 def atom_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
     return int(lib().atom_gemm_workspace_bytes(M, N, K))
+
+
+def atom_probe_mma_i8(groups: int, stream=None) -> int:
+    """Measurement aid: launches the INT8 tensor-core peak loop (see
+    include/atom.h) and returns the integer operations it performs."""
+    pairs = ct.c_int32(0)
+    _check("atom_probe_mma_i8", lib().atom_probe_mma_i8(groups, ct.byref(pairs), _stream(stream)))
+    return 2 * 256 * 256 * 128 * groups * pairs.value
+
+
+def atom_debug_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Test aid: runs the library's bounded mbarrier wait on a barrier nothing
+    arrives on, with a limit of `limit_ns`; the wait gives up and the device
+    status becomes ATOM_ERR_TIMEOUT (see include/atom.h)."""
+    _check("atom_debug_wait_timeout", lib().atom_debug_wait_timeout(limit_ns, _stream(stream)))
 
 
 def atom_device_status(clear: bool = True) -> int:

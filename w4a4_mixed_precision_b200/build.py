@@ -14,7 +14,8 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = [os.path.join(CSRC, f) for f in ("atom_lib.cu", "ptx.cuh", "quant.cuh", "gemm.cuh")]
+# every source of the library: a change to any of them makes the .so stale
+SOURCES = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh")))
 HEADER = os.path.join(ROOT, "include", "atom.h")
 LIB = os.path.join(PKG, "libatom_b200.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -1,6 +1,7 @@
 // atom_lib.cu -- the C ABI declared in include/atom.h: host-side argument
 // checks, tensor-map encoding and kernel launches. No allocation, no host
 // synchronisation on any compute entry point.
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -11,6 +12,7 @@
 #include "ptx.cuh"
 #include "quant.cuh"
 #include "kv.cuh"
+#include "probe.cuh"
 #include "w8a8.cuh"
 
 namespace {
@@ -18,18 +20,21 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxK = atomk::kQuantMaxK;  // gather offsets are uint16 in shared memory
 
+// Per-device launch facts, filled once. The flags that publish a field read
+// outside g_mutex are atomics (written with release after the field, read with
+// acquire); everything else is only touched under g_mutex.
 struct DeviceState {
-  bool probed = false;
+  std::atomic<bool> probed{false};   // publishes supported, sm_count, smem_optin
   bool supported = false;
   int sm_count = 0;
   int smem_optin = 0;
-  bool gemm_attr[6] = {};        // by GEMM kernel: mode (Y, partials, quantized Y) + 3 * W4A8
+  std::atomic<bool> gemm_attr[6] = {};   // by GEMM kernel: mode (Y, partials, quantized Y) + 3 * W4A8
   int gemm_clusters[6] = {};     // co-resident CTA pairs of the GEMM kernel
   bool small_attr = false;       // shared-memory limit set for the small-M GEMM kernels
   bool w8a8_attr = false;
   int w8a8_clusters = 0;          // co-resident CTA pairs of the W8A8 kernel
   uint32_t quant_smem_set = 0;
-  void *noalloc_scratch = nullptr;  // device address of g_noalloc_scratch on this device
+  std::atomic<void *> noalloc_scratch{nullptr};  // device address of g_noalloc_scratch here
 };
 
 DeviceState g_devices[kMaxDevices];
@@ -39,9 +44,9 @@ atom_status_t current_device(DeviceState **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATOM_ERR_CUDA;
   DeviceState &d = g_devices[dev];
-  if (!d.probed) {
+  if (!d.probed.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (!d.probed) {
+    if (!d.probed.load(std::memory_order_relaxed)) {
       int major = 0, minor = 0;
       if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
           cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -50,7 +55,7 @@ atom_status_t current_device(DeviceState **out) {
               cudaSuccess)
         return ATOM_ERR_CUDA;
       d.supported = (major == 10 && minor == 0);  // built for sm_100a only
-      d.probed = true;
+      d.probed.store(true, std::memory_order_release);
     }
   }
   if (!d.supported) return ATOM_ERR_UNSUPPORTED;
@@ -190,13 +195,15 @@ int small_splits(int64_t N, int64_t K, int sms) {
 }
 
 // The GEMM for M <= 64 tokens: weights on the MMA's M side (see gemm_small.cuh).
+// With `partials` (the debug entry point) K is never split.
 atom_status_t launch_gemm_small(DeviceState *dev, const uint8_t *qa4, const int8_t *qa8,
                                 const float *sa, const uint8_t *qw4, const int8_t *qw8,
-                                const float *sw, void *y, int64_t M, int64_t N, int64_t K,
-                                void *workspace, size_t workspace_bytes, atom_stream_t stream) {
+                                const float *sw, void *y, int32_t *partials, int64_t M,
+                                int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                                atom_stream_t stream) {
   using namespace atomk::small_cfg;
   const int64_t q4_row = (K - 128) / 2;
-  int splits = small_splits(N, K, dev->sm_count);
+  int splits = partials != nullptr ? 1 : small_splits(N, K, dev->sm_count);
   if (splits > 1 && (workspace == nullptr ||
                      workspace_bytes < static_cast<size_t>(splits) * M * N * sizeof(float) ||
                      !aligned(workspace, 16)))
@@ -204,9 +211,13 @@ atom_status_t launch_gemm_small(DeviceState *dev, const uint8_t *qa4, const int8
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!dev->small_attr) {
-      const void *fns[3] = {reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<16>),
-                            reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<32>),
-                            reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<64>)};
+      const void *fns[6] = {
+          reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<16>),
+          reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<32>),
+          reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<64>),
+          reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<16, true>),
+          reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<32, true>),
+          reinterpret_cast<const void *>(atomk::w4a4_gemm_small_kernel<64, true>)};
       for (const void *fn : fns)
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kSmemBytes)) != cudaSuccess)
@@ -226,6 +237,7 @@ atom_status_t launch_gemm_small(DeviceState *dev, const uint8_t *qa4, const int8
   p.sa = sa;
   p.sw = sw;
   p.y = static_cast<__half *>(y);
+  p.partials = partials;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
@@ -249,12 +261,20 @@ atom_status_t launch_gemm_small(DeviceState *dev, const uint8_t *qa4, const int8
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   cudaError_t err;
-  if (M <= 16)
+  if (partials != nullptr) {
+    if (M <= 16)
+      err = cudaLaunchKernelEx(&cfg, atomk::w4a4_gemm_small_kernel<16, true>, maps, p);
+    else if (M <= 32)
+      err = cudaLaunchKernelEx(&cfg, atomk::w4a4_gemm_small_kernel<32, true>, maps, p);
+    else
+      err = cudaLaunchKernelEx(&cfg, atomk::w4a4_gemm_small_kernel<64, true>, maps, p);
+  } else if (M <= 16) {
     err = cudaLaunchKernelEx(&cfg, atomk::w4a4_gemm_small_kernel<16>, maps, p);
-  else if (M <= 32)
+  } else if (M <= 32) {
     err = cudaLaunchKernelEx(&cfg, atomk::w4a4_gemm_small_kernel<32>, maps, p);
-  else
+  } else {
     err = cudaLaunchKernelEx(&cfg, atomk::w4a4_gemm_small_kernel<64>, maps, p);
+  }
   return err == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
 }
 
@@ -290,8 +310,9 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   using namespace atomk::gemm_cfg;
   const bool pmode = partials != nullptr;
   const int mode = pmode ? kModePartials : (qmode ? kModeQuantY : kModeY);
-  if (mode == kModeY && !a8 && M <= atomk::small_cfg::kMaxTokens)
-    return launch_gemm_small(dev, qa4, qa8, sa, qw4, qw8, sw, y, M, N, K, workspace,
+  // A few tokens (decode): the small-M kernel, for Y and for the partials alike.
+  if ((mode == kModeY || mode == kModePartials) && !a8 && M <= atomk::small_cfg::kMaxTokens)
+    return launch_gemm_small(dev, qa4, qa8, sa, qw4, qw8, sw, y, partials, M, N, K, workspace,
                              workspace_bytes, stream);
   int pairs = 0;
   if ((st = gemm_pairs(dev, mode + (a8 ? 3 : 0), &pairs)) != ATOM_OK) return st;
@@ -382,8 +403,12 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
 // Co-resident CTA pairs of the GEMM kernel on this device (cached per device).
 atom_status_t gemm_pairs(DeviceState *dev, int mode, int *pairs) {
   using namespace atomk::gemm_cfg;
-  if (!dev->gemm_attr[mode]) {
+  if (!dev->gemm_attr[mode].load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lock(g_mutex);
+    if (dev->gemm_attr[mode].load(std::memory_order_relaxed)) {
+      *pairs = dev->gemm_clusters[mode];
+      return ATOM_OK;
+    }
     const void *fn =
         mode == kModePartials ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<true>)
         : mode == kModeQuantY ? reinterpret_cast<const void *>(atomk::w4a4_gemm_kernel<false, true>)
@@ -410,9 +435,27 @@ atom_status_t gemm_pairs(DeviceState *dev, int mode, int *pairs) {
     if (cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg) != cudaSuccess || clusters < 1)
       clusters = dev->sm_count / 2;
     dev->gemm_clusters[mode] = clusters;
-    dev->gemm_attr[mode] = true;
+    dev->gemm_attr[mode].store(true, std::memory_order_release);
   }
   *pairs = dev->gemm_clusters[mode];
+  return ATOM_OK;
+}
+
+// Workspace bytes atom_w4a4_gemm asks for on this shape: splits * M * N * 4
+// when the kernel that will run (the small-M kernel for M <= 64, the large
+// one otherwise) would split K, else 0.
+atom_status_t gemm_workspace_need(DeviceState *dev, int64_t M, int64_t N, int64_t K,
+                                  size_t *bytes) {
+  int splits = 1;
+  if (M <= atomk::small_cfg::kMaxTokens) {
+    splits = small_splits(N, K, dev->sm_count);
+  } else {
+    int pairs = 0;
+    const atom_status_t st = gemm_pairs(dev, kModeY, &pairs);
+    if (st != ATOM_OK) return st;
+    splits = gemm_splits(M, N, K, pairs);
+  }
+  *bytes = splits > 1 ? static_cast<size_t>(splits) * M * N * sizeof(float) : 0;
   return ATOM_OK;
 }
 
@@ -602,16 +645,9 @@ atom_status_t atom_w4a4_gemm_quant(const uint8_t *qa4, const int8_t *qa8, const 
 size_t atom_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K < 256) return 0;
   DeviceState *dev = nullptr;
-  int pairs = 0;
   if (current_device(&dev) != ATOM_OK) return 0;
-  int splits = 1;
-  if (M <= atomk::small_cfg::kMaxTokens) {
-    splits = small_splits(N, K, dev->sm_count);
-  } else {
-    if (gemm_pairs(dev, kModeY, &pairs) != ATOM_OK) return 0;
-    splits = gemm_splits(M, N, K, pairs);
-  }
-  return splits > 1 ? static_cast<size_t>(splits) * M * N * sizeof(float) : 0;
+  size_t bytes = 0;
+  return gemm_workspace_need(dev, M, N, K, &bytes) == ATOM_OK ? bytes : 0;
 }
 
 atom_status_t atom_device_status(int clear) {
@@ -625,6 +661,49 @@ atom_status_t atom_device_status(int clear) {
       return ATOM_ERR_CUDA;
   }
   return static_cast<atom_status_t>(v);
+}
+
+atom_status_t atom_probe_mma_i8(int64_t groups, int32_t *pairs_out, atom_stream_t stream) {
+  if (groups < 1 || groups > (int64_t(1) << 20) || pairs_out == nullptr) return ATOM_ERR_INVALID_ARG;
+  DeviceState *dev = nullptr;
+  atom_status_t st = current_device(&dev);
+  if (st != ATOM_OK) return st;
+  using namespace atomk::probe_cfg;
+  int pairs = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    const void *fn = reinterpret_cast<const void *>(atomk::mma_i8_probe_kernel);
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+      return ATOM_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * dev->sm_count, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&pairs, fn, &cfg) != cudaSuccess || pairs < 1)
+      pairs = dev->sm_count / 2;
+  }
+  atomk::mma_i8_probe_kernel<<<2 * pairs, kThreads, kSmemBytes,
+                               reinterpret_cast<cudaStream_t>(stream)>>>(groups);
+  if (cudaGetLastError() != cudaSuccess) return ATOM_ERR_CUDA;
+  *pairs_out = pairs;
+  return ATOM_OK;
+}
+
+atom_status_t atom_debug_wait_timeout(uint64_t limit_ns, atom_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > atomk::kWaitLimitNs) return ATOM_ERR_INVALID_ARG;
+  DeviceState *dev = nullptr;
+  const atom_status_t st = current_device(&dev);
+  if (st != ATOM_OK) return st;
+  atomk::wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
 }
 
 const char *atom_status_string(atom_status_t status) {
@@ -646,13 +725,13 @@ int atom_version(void) { return 100; }
 
 // ---------------------------------------------------------------- allocation-free GEMM
 //
-// Some callers cannot allocate device memory around a GEMM call: code that
-// runs while a CUDA graph is being captured (an allocation there is not part
-// of the graph and breaks replay), serving runtimes that hand every byte of
-// device memory to a fixed pool at start-up, and C callers with no device
-// allocator of their own. atom_w4a4_gemm needs scratch only when it splits K
-// (small M), and takes it from the caller. This entry point takes it instead
-// from a fixed array in the library's device memory.
+// Some callers cannot allocate device memory around a GEMM call: serving
+// runtimes that hand every byte of device memory to a fixed pool at start-up
+// (nothing is left to allocate from, and a stray allocation would fragment the
+// pool), and C or embedded callers that have no device allocator of their own.
+// atom_w4a4_gemm needs scratch only when it splits K (M > 64 with few output
+// tiles), and takes it from the caller. This entry point takes it instead from
+// a fixed array in the library's device memory.
 
 namespace {
 
@@ -665,16 +744,17 @@ __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(
 // g_noalloc_scratch is a host-side stand-in, not a device address, so the
 // address is looked up once per device, with that device current.
 atom_status_t noalloc_scratch(DeviceState *dev, void **out) {
-  if (dev->noalloc_scratch == nullptr) {
+  void *p = dev->noalloc_scratch.load(std::memory_order_acquire);
+  if (p == nullptr) {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (dev->noalloc_scratch == nullptr) {
-      void *p = nullptr;
+    p = dev->noalloc_scratch.load(std::memory_order_relaxed);
+    if (p == nullptr) {
       if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
         return ATOM_ERR_CUDA;
-      dev->noalloc_scratch = p;
+      dev->noalloc_scratch.store(p, std::memory_order_release);
     }
   }
-  *out = dev->noalloc_scratch;
+  *out = p;
   return ATOM_OK;
 }
 
@@ -689,13 +769,14 @@ extern "C" ATOM_API atom_status_t atom_w4a4_gemm_noalloc(
   if (st != ATOM_OK) return st;
   if (M == 0) return ATOM_OK;
   if (!y) return ATOM_ERR_INVALID_ARG;
+  if (N < 8 || N % 8 != 0 || M > INT32_MAX || N > INT32_MAX) return ATOM_ERR_SHAPE;
   DeviceState *dev = nullptr;
   if ((st = current_device(&dev)) != ATOM_OK) return st;
-  int pairs = 0;
-  if ((st = gemm_pairs(dev, kModeY, &pairs)) != ATOM_OK) return st;
-  const int splits = gemm_splits(M, N, K, pairs);
-  if (splits > 1 &&
-      static_cast<double>(splits) * M * N * sizeof(float) > static_cast<double>(kNoAllocScratchBytes))
+  // the scratch the split of the kernel that will run needs (the same rule as
+  // atom_gemm_workspace_bytes)
+  size_t need = 0;
+  if ((st = gemm_workspace_need(dev, M, N, K, &need)) != ATOM_OK) return st;
+  if (need > kNoAllocScratchBytes)
     return ATOM_ERR_SHAPE;   // the split's partial tiles do not fit in the fixed scratch
   void *scratch = nullptr;
   if ((st = noalloc_scratch(dev, &scratch)) != ATOM_OK) return st;

@@ -73,7 +73,8 @@ struct SmallMaps {
 struct SmallParams {
   const float *sa;   // [G][M]
   const float *sw;   // [G][N]
-  __half *y;
+  __half *y;         // may be null in partials mode
+  int32_t *partials; // partials mode only: int32 [G][M][N]
   int M, N, K, G;
   int n_tiles, splits, items;   // splits > 1: one item per CTA, a cluster of `splits` CTAs per tile
 };
@@ -111,7 +112,11 @@ __device__ __forceinline__ int64_t small_iterations(const SmallParams &p) {
   return n;
 }
 
-template <int NT>
+// kPartials: also write each group's exact int32 partial sums P[g][m][n] (the
+// debug entry point), read from the biased accumulator before the scale
+// arithmetic: P = (bits - bias) >> 8 for an INT4 group (the tiles hold 16*q, so
+// the MMA sums 256*P), bits - bias for the INT8 group.
+template <int NT, bool kPartials = false>
 __global__ void __launch_bounds__(small_cfg::kThreads, 1)
 w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams p) {
   using namespace small_cfg;
@@ -221,6 +226,19 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
         uint32_t(&r)[16] = (c & 1) ? rb : ra;
         uint32_t(&rn)[16] = (c & 1) ? ra : rb;
         if (c + 1 < NT / 16) tmem_ld_x16(tcol + 16 * (c + 1), rn);
+        if (kPartials) {
+          // weight row n, tokens 16c .. 16c+15; consecutive lanes write
+          // consecutive n of one token row
+          const int n = w.n0 + lrow;
+          const int sh = w.g < p.G - 1 ? 8 : 0;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int m = 16 * c + e;
+            if (n < p.N && m < p.M)
+              p.partials[(static_cast<int64_t>(w.g) * p.M + m) * p.N + n] =
+                  static_cast<int32_t>(r[e] - gemm_cfg::kBias) >> sh;
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {   // token pair 8c + j: columns 16c + 2j, 16c + 2j + 1
           const float4 s4 = sap[8 * c + j];
@@ -256,7 +274,7 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
             const float v = h ? acc[j].y : acc[j].x;
             if (p.splits > 1)
               part[m * BW + lrow] = v;
-            else if (row_ok && m < p.M)
+            else if (row_ok && m < p.M && p.y != nullptr)
               p.y[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(v);
           }
           acc[j] = make_float2(0.f, 0.f);

@@ -66,17 +66,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Slow path of mbar_wait: keeps polling, and gives up after kWaitLimitNs or
-// once `abort_flag` (shared memory) becomes non-zero. Kept out of line so that
-// the timer read never lands on the fast path.
+// Slow path of mbar_wait: keeps polling, and gives up after `limit_ns`
+// (kWaitLimitNs in every kernel of the library) or once `abort_flag` (shared
+// memory) becomes non-zero. Kept out of line so that the timer read never
+// lands on the fast path.
 __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity,
-                                            const volatile int *abort_flag) {
+                                            const volatile int *abort_flag,
+                                            uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
       if (abort_flag != nullptr && *abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+      if (global_timer_ns() - t0 > limit_ns) return false;
     }
   }
 }
@@ -539,6 +541,21 @@ __device__ int g_device_status;
 
 __device__ __forceinline__ void report_status(int code) {
   atomicCAS(&g_device_status, 0, code);
+}
+
+// Exercises the bounded-wait path that every pipeline wait of the library
+// takes when a phase does not complete: one thread waits, through
+// mbar_wait/mbar_wait_slow, on an mbarrier that nothing arrives on and no copy
+// or MMA is tied to, gives up after `limit_ns`, and records ATOM_ERR_TIMEOUT
+// (6) in the status word exactly as the GEMM and quantizer kernels do. Nothing
+// is in flight when it returns, so the context stays usable.
+__global__ void wait_timeout_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  if (!mbar_try_wait(&bar, 0) && !mbar_wait_slow(&bar, 0, nullptr, limit_ns))
+    report_status(6 /* ATOM_ERR_TIMEOUT */);
 }
 
 }  // namespace atomk
