@@ -251,6 +251,50 @@ ATOM_API atom_status_t atom_w4a4_gemm_quant(const uint8_t *qa4, const int8_t *qa
                                            atom_stream_t stream);
 
 /*
+ * Tiled weight layout -- the library's own layout of the packed INT4 weight
+ * codes, a one-off repack of what atom_quant_weights writes.
+ *
+ * The pages fix what the codes are (4-bit groups of 128 channels with per-group
+ * scales: "Atom (mixed-precision block-outlier low-bit quantization for
+ * serving)", fields Bits and Weight group size; the paper summary's weight
+ * blocks) but not how the weights are laid out for the kernels; the weights
+ * are quantized offline, so their layout is the kernels' choice. In the row
+ * layout qw4 [N][(K-128)/2], the 128-row x 64-byte piece a GEMM needs per
+ * weight tile and group is 128 pieces of 64 bytes, (K-128)/2 bytes apart. The
+ * tiled layout stores each (tile, group) piece as one contiguous 8 KB block:
+ *
+ *   qw4t[((t * G4 + g) * 128 + r) * 64 + j] = qw4[128 t + r][64 g + j]
+ *   for tile t < ceil(N/128), group g < G4 = K/128 - 1, row r < 128, j < 64;
+ *   rows 128 t + r >= N of the last tile are zero.
+ *
+ * qw8 and sw keep their layouts. A decode GEMM reads every weight once per
+ * call, and reads the tiled layout as long contiguous runs instead of 64-byte
+ * pieces.
+ *
+ * atom_tiled_weights_bytes: bytes of the tiled layout, ceil(N/128) * G4 * 8192
+ *   (0 for N <= 0 or a K outside [256, 32768] or not a multiple of 128).
+ * atom_pack_weights_tiled: qw4 (row layout, N rows) -> qw4t (tiled layout).
+ * atom_unpack_weights_tiled: qw4t -> qw4 (rows n < N), the inverse copy.
+ *   N >= 0 (0 is a no-op), K as for atom_quant_weights; both pointers device
+ *   memory, 16-byte aligned; the buffers must not overlap.
+ * atom_w4a4_gemm_tiled: atom_w4a4_gemm (same arguments, result and errors) with
+ *   the packed INT4 weights `qw4t` in the tiled layout. Same kernels, same
+ *   arithmetic in the same order: Y is bit-identical to atom_w4a4_gemm's on the
+ *   row layout of the same weights, with the same workspace.
+ */
+ATOM_API size_t atom_tiled_weights_bytes(int64_t N, int64_t K);
+ATOM_API atom_status_t atom_pack_weights_tiled(const uint8_t *qw4, int64_t N, int64_t K,
+                                               uint8_t *qw4t, atom_stream_t stream);
+ATOM_API atom_status_t atom_unpack_weights_tiled(const uint8_t *qw4t, int64_t N, int64_t K,
+                                                 uint8_t *qw4, atom_stream_t stream);
+ATOM_API atom_status_t atom_w4a4_gemm_tiled(const uint8_t *qa4, const int8_t *qa8,
+                                            const float *sa, const uint8_t *qw4t,
+                                            const int8_t *qw8, const float *sw, void *y,
+                                            int64_t M, int64_t N, int64_t K, int32_t n_outlier,
+                                            int32_t group, void *workspace,
+                                            size_t workspace_bytes, atom_stream_t stream);
+
+/*
  * Bytes of workspace atom_w4a4_gemm uses for this shape on the current device:
  * splits * M * N * 4 when it would split K, else 0 (also 0 on error).
  */

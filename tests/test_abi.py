@@ -206,3 +206,25 @@ def test_timeout_aid_validates_its_limit_on_the_host(lib):
     production 1 s before touching the device."""
     assert lib.atom_debug_wait_timeout(0, None) == INVALID
     assert lib.atom_debug_wait_timeout(2_000_000_000, None) == INVALID
+
+
+def test_tiled_layout_entry_points_check_arguments_on_the_host(lib):
+    assert lib.atom_tiled_weights_bytes(264, 1152) == 3 * 8 * 8192
+    assert lib.atom_tiled_weights_bytes(0, 1152) == 0
+    assert lib.atom_tiled_weights_bytes(264, 1000) == 0
+    for fn in (lib.atom_pack_weights_tiled, lib.atom_unpack_weights_tiled):
+        assert fn(A16, 0, 512, A16, None) == OK          # nothing to do
+        assert fn(A16, -1, 512, A16, None) == INVALID
+        assert fn(A16, 16, 500, A16, None) == SHAPE
+        assert fn(A16, 16, 128, A16, None) == SHAPE
+        assert fn(0, 16, 512, A16, None) == INVALID
+        assert fn(A16, 16, 512, 0, None) == INVALID
+        assert fn(MIS, 16, 512, A16, None) == ALIGN
+        assert fn(A16, 16, 512, A16 + 8, None) == ALIGN
+    g = lib.atom_w4a4_gemm_tiled
+    args = [A16] * 6
+    assert g(*args, A16, 0, 256, 512, 128, 128, None, 0, None) == OK
+    assert g(*args, 0, 16, 256, 512, 128, 128, None, 0, None) == INVALID    # no y
+    assert g(*args, A16, 16, 260, 512, 128, 128, None, 0, None) == SHAPE    # N % 8 != 0
+    assert g(A16, A16, A16, MIS, A16, A16, A16, 16, 256, 512, 128, 128, None, 0, None) == ALIGN
+    assert g(*args, A16, 16, 256, 512, 64, 128, None, 0, None) == UNSUPPORTED

@@ -59,6 +59,14 @@ SIGNATURES = {
     "atom_w4a4_gemm_quant": ([ct.c_void_p] * 6 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_int32,
                               ct.c_int32] + [ct.c_void_p] * 4, ct.c_int),
     "atom_gemm_workspace_bytes": ([ct.c_int64, ct.c_int64, ct.c_int64], ct.c_size_t),
+    "atom_tiled_weights_bytes": ([ct.c_int64, ct.c_int64], ct.c_size_t),
+    "atom_pack_weights_tiled": ([ct.c_void_p, ct.c_int64, ct.c_int64, ct.c_void_p, ct.c_void_p],
+                                ct.c_int),
+    "atom_unpack_weights_tiled": ([ct.c_void_p, ct.c_int64, ct.c_int64, ct.c_void_p, ct.c_void_p],
+                                  ct.c_int),
+    "atom_w4a4_gemm_tiled": ([ct.c_void_p] * 7 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_int32,
+                                                  ct.c_int32, ct.c_void_p, ct.c_size_t,
+                                                  ct.c_void_p], ct.c_int),
     "atom_w4a4_gemm_noalloc": ([ct.c_void_p] * 7 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_int32,
                                                     ct.c_int32, ct.c_void_p], ct.c_int),
     "atom_w8a8_gemm": ([ct.c_void_p] * 5 + [ct.c_int64, ct.c_int64, ct.c_int64, ct.c_void_p],
@@ -294,6 +302,78 @@ def atom_w4a4_gemm(qa: Quantized, qw: Quantized, K: int, y: Optional[torch.Tenso
         _dev(y, torch.float16, "y"), M, N, K, N_OUTLIER, GROUP, ws_ptr, ws_bytes, _stream(stream))
     _check("atom_w4a4_gemm", st)
     return y
+
+
+class TiledWeights(NamedTuple):
+    """Quantized weights with the INT4 codes in the tiled layout (see
+    include/atom.h): q4t uint8 [ceil(N/128), K/128 - 1, 128, 64]; q8 and scales as
+    in Quantized."""
+    q4t: torch.Tensor
+    q8: torch.Tensor
+    scales: torch.Tensor
+
+    @property
+    def rows(self) -> int:
+        return self.q8.shape[0]
+
+
+def _tiled_shape(N: int, K: int):
+    return ((N + 127) // 128, K // GROUP - 1, 128, 64)
+
+
+def atom_pack_weights_tiled(qw: Quantized, K: int, stream=None) -> TiledWeights:
+    """One-off repack of quantized weights into the tiled layout."""
+    N = qw.rows
+    _check_quantized(qw, K, "qw")
+    q4t = torch.empty(_tiled_shape(N, K), dtype=torch.uint8, device=qw.q4.device)
+    st = lib().atom_pack_weights_tiled(_dev(qw.q4, torch.uint8, "qw4"), N, K,
+                                       _dev(q4t, torch.uint8, "qw4t"), _stream(stream))
+    _check("atom_pack_weights_tiled", st)
+    return TiledWeights(q4t, qw.q8, qw.scales)
+
+
+def atom_unpack_weights_tiled(qwt: TiledWeights, K: int, stream=None) -> torch.Tensor:
+    """The row layout [N, (K-128)/2] of tiled INT4 weight codes (the inverse repack)."""
+    N = qwt.rows
+    if _valid_k(K):
+        _expect_shape(qwt.q4t, _tiled_shape(N, K), "qw4t")
+    q4 = torch.empty((N, (K - N_OUTLIER) // 2), dtype=torch.uint8, device=qwt.q4t.device)
+    st = lib().atom_unpack_weights_tiled(_dev(qwt.q4t, torch.uint8, "qw4t"), N, K,
+                                         _dev(q4, torch.uint8, "qw4"), _stream(stream))
+    _check("atom_unpack_weights_tiled", st)
+    return q4
+
+
+def atom_w4a4_gemm_tiled(qa: Quantized, qwt: TiledWeights, K: int,
+                         y: Optional[torch.Tensor] = None, stream=None,
+                         workspace: Optional[torch.Tensor] = None,
+                         split: bool = True) -> torch.Tensor:
+    """atom_w4a4_gemm with the weights in the tiled layout (bit-identical Y)."""
+    M, N = qa.rows, qwt.rows
+    dev = qa.q4.device
+    _check_quantized(qa, K, "qa")
+    if _valid_k(K):
+        _expect_shape(qwt.q4t, _tiled_shape(N, K), "qw4t")
+        _expect_shape(qwt.q8, (N, N_OUTLIER), "qw.q8")
+        _expect_shape(qwt.scales, (K // GROUP, N), "qw.scales")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    _expect_shape(y, (M, N), "y")
+    if workspace is None and split:
+        workspace = gemm_workspace(M, N, K, dev)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None or not split else (
+        _dev(workspace, torch.uint8, "workspace"), workspace.numel())
+    st = lib().atom_w4a4_gemm_tiled(
+        _dev(qa.q4, torch.uint8, "qa4"), _dev(qa.q8, torch.int8, "qa8"),
+        _dev(qa.scales, torch.float32, "sa"), _dev(qwt.q4t, torch.uint8, "qw4t"),
+        _dev(qwt.q8, torch.int8, "qw8"), _dev(qwt.scales, torch.float32, "sw"),
+        _dev(y, torch.float16, "y"), M, N, K, N_OUTLIER, GROUP, ws_ptr, ws_bytes, _stream(stream))
+    _check("atom_w4a4_gemm_tiled", st)
+    return y
+
+
+def atom_tiled_weights_bytes(N: int, K: int) -> int:
+    return int(lib().atom_tiled_weights_bytes(N, K))
 
 
 def atom_w4a4_gemm_noalloc(qa: Quantized, qw: Quantized, K: int,

@@ -13,6 +13,7 @@
 #include "quant.cuh"
 #include "kv.cuh"
 #include "probe.cuh"
+#include "tiled.cuh"
 #include "w8a8.cuh"
 
 namespace {
@@ -200,7 +201,7 @@ atom_status_t launch_gemm_small(DeviceState *dev, const uint8_t *qa4, const int8
                                 const float *sa, const uint8_t *qw4, const int8_t *qw8,
                                 const float *sw, void *y, int32_t *partials, int64_t M,
                                 int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
-                                atom_stream_t stream) {
+                                atom_stream_t stream, bool w_tiled) {
   using namespace atomk::small_cfg;
   const int64_t q4_row = (K - 128) / 2;
   int splits = partials != nullptr ? 1 : small_splits(N, K, dev->sm_count);
@@ -227,17 +228,26 @@ atom_status_t launch_gemm_small(DeviceState *dev, const uint8_t *qa4, const int8
   }
   atomk::SmallMaps maps;
   const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  if (!encode_2d(&maps.w4, u8, qw4, q4_row, N, q4_row, 64, BW, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+  // the INT8 group comes in two halves (64 W rows + 32 token rows each)
+  // (tiled W: bulk copies of qw4's blocks, no W4 tensor map; the slot is
+  // filled with the A4 map, which the kernel then never reads for W)
+  if (!encode_2d(&maps.w4, u8, w_tiled ? static_cast<const void *>(qa4) : qw4, q4_row,
+                 w_tiled ? M : N, q4_row, 64, w_tiled ? kMaxTokens : BW,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !encode_2d(&maps.a4, u8, qa4, q4_row, M, q4_row, 64, kMaxTokens,
                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_2d(&maps.w8, u8, qw8, 128, N, 128, 128, BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&maps.a8, u8, qa8, 128, M, 128, 128, kMaxTokens, CU_TENSOR_MAP_SWIZZLE_128B))
+      !encode_2d(&maps.w8, u8, qw8, 128, N, 128, 128, BW / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&maps.a8, u8, qa8, 128, M, 128, 128, kMaxTokens / 2,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&maps.sw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, sw, N, K / 128, N * 4, BW, 1,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
     return ATOM_ERR_CUDA;
   atomk::SmallParams p;
   p.sa = sa;
   p.sw = sw;
   p.y = static_cast<__half *>(y);
   p.partials = partials;
+  p.qw4t = w_tiled ? qw4 : nullptr;
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
@@ -250,7 +260,8 @@ atom_status_t launch_gemm_small(DeviceState *dev, const uint8_t *qa4, const int8
   const int grid = p.items < dev->sm_count ? p.items : dev->sm_count;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  const int nt = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  cfg.blockDim = dim3(threads_for(nt), 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr;
@@ -283,7 +294,7 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
                           int32_t *partials, int64_t M, int64_t N, int64_t K, int32_t n_outlier,
                           int32_t group, void *workspace, size_t workspace_bytes,
                           atom_stream_t stream, uint8_t *qy4 = nullptr, int8_t *qy8 = nullptr,
-                          float *sy = nullptr, bool a8 = false) {
+                          float *sy = nullptr, bool a8 = false, bool w_tiled = false) {
   if (M < 0 || N < 0) return ATOM_ERR_INVALID_ARG;
   atom_status_t st = check_method_params(K, n_outlier, group);
   if (st != ATOM_OK) return st;
@@ -313,7 +324,7 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   // A few tokens (decode): the small-M kernel, for Y and for the partials alike.
   if ((mode == kModeY || mode == kModePartials) && !a8 && M <= atomk::small_cfg::kMaxTokens)
     return launch_gemm_small(dev, qa4, qa8, sa, qw4, qw8, sw, y, partials, M, N, K, workspace,
-                             workspace_bytes, stream);
+                             workspace_bytes, stream, w_tiled);
   int pairs = 0;
   if ((st = gemm_pairs(dev, mode + (a8 ? 3 : 0), &pairs)) != ATOM_OK) return st;
 
@@ -325,7 +336,9 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   // W4A8: INT8 activations [M][K], one 128-byte box per row and group; no INT4 A
   if (!encode_2d(&maps.a4, u8, a8 ? static_cast<const void *>(qa8) : qa4, q4_row, M, q4_row, 64,
                  BM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !encode_2d(&maps.w4, u8, qw4, q4_row, N, q4_row, 64, BW, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_2d(&maps.w4, u8, w_tiled ? static_cast<const void *>(qa8) : qw4,
+                 w_tiled ? 128 : q4_row, w_tiled ? M : N, w_tiled ? 128 : q4_row, 64, BW,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||   // (tiled W: bulk copies, this map is unused)
       !encode_2d(&maps.a8, u8, qa8, a8 ? K : 128, M, a8 ? K : 128, 128, BM,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&maps.w8, u8, qw8, 128, N, 128, 128, BW, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -360,6 +373,8 @@ atom_status_t launch_gemm(const uint8_t *qa4, const int8_t *qa8, const float *sa
   p.K = static_cast<int>(K);
   p.G = static_cast<int>(G);
   p.sa_by_tma = sa_by_tma ? 1 : 0;
+  p.qw4t = w_tiled ? qw4 : nullptr;
+  p.w_tiles = static_cast<int>((N + BW - 1) / BW);
   p.m_tiles = static_cast<int>((M + kPairM - 1) / kPairM);
   p.n_tiles = static_cast<int>((N + BN - 1) / BN);
   const int64_t tiles = static_cast<int64_t>(p.m_tiles) * p.n_tiles;
@@ -640,6 +655,57 @@ atom_status_t atom_w4a4_gemm_quant(const uint8_t *qa4, const int8_t *qa8, const 
   if ((!qy4 || !qy8 || !sy) && M > 0) return ATOM_ERR_INVALID_ARG;
   return launch_gemm(qa4, qa8, sa, qw4, qw8, sw, nullptr, nullptr, M, N, K, n_outlier, group,
                      nullptr, 0, stream, qy4, qy8, sy);
+}
+
+size_t atom_tiled_weights_bytes(int64_t N, int64_t K) {
+  if (N <= 0 || K % 128 != 0 || K < 256 || K > kMaxK) return 0;
+  return static_cast<size_t>((N + atomk::kTileRows - 1) / atomk::kTileRows) *
+         static_cast<size_t>(K / 128 - 1) * atomk::kTileBlock;
+}
+
+static atom_status_t tiled_copy(const uint8_t *src, int64_t N, int64_t K, uint8_t *dst,
+                                atom_stream_t stream, bool pack) {
+  if (N < 0) return ATOM_ERR_INVALID_ARG;
+  if (K % 128 != 0 || K < 256 || K > kMaxK || N > INT32_MAX) return ATOM_ERR_SHAPE;
+  if (N == 0) return ATOM_OK;
+  if (!src || !dst) return ATOM_ERR_INVALID_ARG;
+  if (!aligned(src, 16) || !aligned(dst, 16)) return ATOM_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  const atom_status_t st = current_device(&dev);
+  if (st != ATOM_OK) return st;
+  const int64_t g4 = K / 128 - 1;
+  const int64_t chunks = static_cast<int64_t>(atom_tiled_weights_bytes(N, K) / 16);
+  int64_t blocks = (chunks + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(dev->sm_count) * 16;
+  if (blocks > cap) blocks = cap;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (pack)
+    atomk::pack_weights_tiled_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(src, dst, N,
+                                                                               (K - 128) / 2, g4, chunks);
+  else
+    atomk::unpack_weights_tiled_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
+        src, dst, N, (K - 128) / 2, g4, chunks);
+  return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
+}
+
+atom_status_t atom_pack_weights_tiled(const uint8_t *qw4, int64_t N, int64_t K, uint8_t *qw4t,
+                                      atom_stream_t stream) {
+  return tiled_copy(qw4, N, K, qw4t, stream, true);
+}
+
+atom_status_t atom_unpack_weights_tiled(const uint8_t *qw4t, int64_t N, int64_t K, uint8_t *qw4,
+                                        atom_stream_t stream) {
+  return tiled_copy(qw4t, N, K, qw4, stream, false);
+}
+
+atom_status_t atom_w4a4_gemm_tiled(const uint8_t *qa4, const int8_t *qa8, const float *sa,
+                                   const uint8_t *qw4t, const int8_t *qw8, const float *sw,
+                                   void *y, int64_t M, int64_t N, int64_t K, int32_t n_outlier,
+                                   int32_t group, void *workspace, size_t workspace_bytes,
+                                   atom_stream_t stream) {
+  if (!y && M > 0) return ATOM_ERR_INVALID_ARG;
+  return launch_gemm(qa4, qa8, sa, qw4t, qw8, sw, y, nullptr, M, N, K, n_outlier, group,
+                     workspace, workspace_bytes, stream, nullptr, nullptr, nullptr, false, true);
 }
 
 size_t atom_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {

@@ -56,8 +56,12 @@
 // starts at the int32 0x4B400000 (the bits of C = 1.5*2^23) and the MMAs add
 // the group's partial P onto it, so the int32 in TMEM is the bit pattern of
 // the float C + P, exact for |P| < 2^22 (INT4 groups: |256 P| <= 1.6e6; INT8
-// group: |P| <= 2.1e6). The drain re-arms its columns with TMEM stores once
-// it has loaded them.
+// group: |P| <= 2.1e6). The bias is written by the tensor core itself: each
+// group starts with one fp16 MMA (K = 16, accumulate off) of two constant
+// tiles whose only nonzero column holds 6144 in A and 2048 in B, so every
+// accumulator element becomes the fp32 6144 * 2048 = 1.5*2^23 exactly, and the
+// group's integer MMAs then accumulate onto those bits. (Re-arming the columns
+// with TMEM stores from the drain cost the drain ~20 % of its time per group.)
 // Dequantisation: with sa' = sa truncated to 22 significant bits, C*sa' is
 // exact for C = 1.5*2^23, so t = fma(F, sa', -C*sa') = round(P*sa') in one
 // instruction, then acc = fma(t, sw, acc); both run as packed f32x2 pairs.
@@ -105,7 +109,14 @@ constexpr uint32_t kSOff = kPOff + kNP * kPSlot;
 // Y staging: one 32-row x 64-column fp16 box (128-byte swizzle) per drain warp
 constexpr uint32_t kYSlot = 32 * 128;
 constexpr uint32_t kYOff = (kSOff + kNS * kSSlot + 1023u) & ~1023u;
-constexpr uint32_t kSmemBytes = kYOff + 8 * kYSlot + 1024;  // + alignment slack
+// bias tiles of the fp16 bias MMA: A then B, each 128 rows x 16 fp16 (K-major,
+// no swizzle: core matrices of 8 rows x 16 B, K-adjacent 128 B apart, row
+// groups 256 B apart)
+constexpr uint32_t kBiasTile = 128 * 32;
+constexpr uint32_t kBiasOff = kYOff + 8 * kYSlot;
+constexpr uint32_t kBiasLbo = 128, kBiasSbo = 256;
+constexpr uint32_t kIdescBias = idesc_f16(2 * 128, 256);
+constexpr uint32_t kSmemBytes = kBiasOff + 2 * kBiasTile + 1024;  // + alignment slack
 constexpr int kPackedChunks = (BM + BW) * 4;                    // 16-B chunks per INT4 group
 constexpr int kChunksPerThread = (kPackedChunks + kUnpackThreads - 1) / kUnpackThreads;
 constexpr int kInt8Chunks = (kABytes + kBBytes) / 16;           // 16-B chunks of an INT8 group
@@ -135,6 +146,8 @@ struct GemmParams {
   int8_t *qy8;         //   INT8 codes of its last 128 columns [M][128],
   float *sy;           //   and group scales [N/128][M]
   float *ws;           // splits > 1: fp32 partial outputs [splits][M][N]
+  const uint8_t *qw4t; // packed INT4 W in the tiled layout (tiled.cuh), or null: row layout by TMA
+  int w_tiles;         // 128-row weight tiles, ceil(N / 128)
   int M, N, K, G;
   int m_tiles, n_tiles, tiles;   // pair tiles of 256 x 256
   int splits;                    // K splits per tile (1: no split)
@@ -384,6 +397,14 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = static_cast<int>(cluster_cta_rank());
 
+  // the bias tiles: element (row, k = 0) = 6144 (A) or 2048 (B), all else 0
+  for (int i = threadIdx.x; i < static_cast<int>(2 * kBiasTile / 16); i += kThreads) {
+    const int t = i / static_cast<int>(kBiasTile / 16), j = (i >> 3) & 1;
+    const uint32_t v = j == 0 ? (t == 0 ? 0x6E00u : 0x6800u) : 0u;   // fp16 6144 / 2048
+    reinterpret_cast<uint4 *>(smem + kBiasOff)[i] = make_uint4(v, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNP; ++s) {
       mbar_init(&pfull[s], 1);       // producer's expect_tx arrival (+ TMA bytes)
@@ -414,20 +435,6 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   tc_fence_after_sync();
   const uint32_t tbase = *tmem_slot;
   const int64_t iters = pair_iterations(p);
-
-  // Both accumulators start at the conversion bias (see the drain), and every
-  // MMA accumulates onto what TMEM holds.
-  if (warp >= 8) {
-    const uint32_t lanes = tbase + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
-                           ((warp - 8) >> 2) * kHalfN;
-#pragma unroll
-    for (int c = 0; c < 64; ++c)   // buffer c/32, 4-column chunk c%32 of this warp's half
-      tmem_st_x4_fill(lanes + (c >> 5) * BN + 4 * (c & 31), kBias);
-    tmem_st_wait();
-  }
-  tc_fence_before_sync();
-  cluster_sync();
-  tc_fence_after_sync();
 
   auto fail = [&](void) {
     report_status(6 /* ATOM_ERR_TIMEOUT */);
@@ -520,12 +527,8 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         }
         if (c + 1 < 8) tmem_ld_wait(rn);
       }
-      // this warp's lanes of the half are in registers: re-arm them with the
-      // bias (in one burst, off the arithmetic's path) and hand them back, and
-      // the group's scales with them
-#pragma unroll
-      for (int e = 0; e < kHalfN / 4; ++e) tmem_st_x4_fill(tcol + 4 * e, kBias);
-      tmem_st_wait();
+      // this warp's lanes of the half are in registers: hand them back (the
+      // next group's bias MMA rewrites them), and the group's scales with them
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) {
@@ -659,13 +662,29 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
               break;
             }
             uint8_t *slot = pring + s * kPSlot;
+            // The packed INT4 W tile: one 8 KB bulk copy from the tiled layout,
+            // or a TMA box of the row layout. A tiled W tile past the last
+            // weight tile (a pair tile that overhangs N by 128 rows or more) is
+            // not fetched: its rows only feed output columns >= N.
+            const int wt = wrow / BW;
+            const bool w_fetch = p.qw4t == nullptr || wt < p.w_tiles;
+            auto load_w4 = [&](uint8_t *dst) {
+              if (p.qw4t != nullptr) {
+                if (w_fetch)
+                  bulk_load(dst, p.qw4t + (static_cast<int64_t>(wt) * (p.G - 1) + wp.g) * (BW * 64),
+                            BW * 64u, &pfull[s]);
+              } else {
+                tma_load_2d(dst, &maps.w4, wp.g * 64, wrow, &pfull[s]);
+              }
+            };
+            const uint32_t w4_bytes = w_fetch ? BW * 64u : 0u;
             if (part == 0) {
-              const uint32_t bytes = (two_slots ? kABytes : (BM + BW) * 64u) + BN * 4u +
+              const uint32_t bytes = (two_slots ? kABytes : BM * 64u + w4_bytes) + BN * 4u +
                                      (p.sa_by_tma ? BM * 4u : 0u);
               mbar_arrive_expect_tx(&pfull[s], bytes);
               if (!two_slots) {
                 tma_load_2d(slot, &maps.a4, wp.g * 64, arow, &pfull[s]);
-                tma_load_2d(slot + kPackWOff, &maps.w4, wp.g * 64, wrow, &pfull[s]);
+                load_w4(slot + kPackWOff);
               } else {
                 // W4A4: the INT8 outlier tile of A ([M][128]); W4A8: group g of A ([M][K])
                 tma_load_2d(slot, &maps.a8, kA8 ? wp.g * 128 : 0, arow, &pfull[s]);
@@ -674,8 +693,8 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
               if (p.sa_by_tma) tma_load_2d(slot + kSaLinOff, &maps.sa, arow, wp.g, &pfull[s]);
             } else if (int4_group) {
               // W4A8: the packed INT4 weight tile in the second slot
-              mbar_arrive_expect_tx(&pfull[s], BW * 64u);
-              tma_load_2d(slot, &maps.w4, wp.g * 64, wrow, &pfull[s]);
+              mbar_arrive_expect_tx(&pfull[s], w4_bytes);
+              load_w4(slot);
             } else {
               mbar_arrive_expect_tx(&pfull[s], kBBytes);
               tma_load_2d(slot, &maps.w8, 0, wrow, &pfull[s]);
@@ -701,6 +720,10 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         int64_t last_mma = -1;
         bool ok = true;
         RingPos ur;
+        const uint64_t bias_adesc =
+            smem_desc_k_noswizzle(smem_addr(smem + kBiasOff), kBiasLbo, kBiasSbo);
+        const uint64_t bias_bdesc =
+            smem_desc_k_noswizzle(smem_addr(smem + kBiasOff + kBiasTile), kBiasLbo, kBiasSbo);
         for (int64_t it = 0; ok && it < iters; ++it, ur.next(kNU)) {
           const int u = ur.idx, b = static_cast<int>(it & 1);
           const uint32_t ph = ur.phase;
@@ -718,6 +741,8 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
           const uint64_t adesc = smem_desc_k_sw128(a_addr);
           const uint64_t bdesc = smem_desc_k_sw128(a_addr + kABytes);
           const uint32_t d = tbase + b * BN;
+          // the group's accumulator starts at the conversion bias (see above)
+          mma_f16_pair(d, bias_adesc, bias_bdesc, kIdescBias, 0u);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_i8_pair(d, adesc + 2 * k, bdesc + 2 * k, kIdesc, 1u);

@@ -11,20 +11,33 @@
 //   one CTA owns 128 weight rows (output columns n0..n0+127) and one range of
 //   K groups; per group, four tcgen05.mma.cta_group::1.kind::i8 with M = 128
 //   (weight rows), N = NT (the tokens rounded up to 16, 32 or 64), K = 32
-//   accumulate into an NT-column TMEM accumulator (two alternate); four drain
-//   warps, one per TMEM lane quarter, hold one weight row each and NT token
-//   columns of fp32 accumulators; K is split so that about one CTA per SM
-//   works. The K ranges of one weight tile are one thread-block cluster (at
-//   most 8 CTAs): each parks its fp32 partial tile in its own shared memory,
-//   and after a cluster barrier every CTA sums a slice of the tile over all
-//   of them through distributed shared memory, in K-range order, with the
-//   same fp32 additions as the ordered split-K reduction of gemm.cuh, and
-//   writes fp16 Y.
+//   accumulate into one of four NT-column TMEM accumulators; K is split so
+//   that about one CTA per SM works. The K ranges of one weight tile are one
+//   thread-block cluster (at most 8 CTAs): each parks its fp32 partial tile in
+//   its own shared memory, and after a cluster barrier every CTA sums a slice
+//   of the tile over all of them through distributed shared memory, in K-range
+//   order, with the same fp32 additions as the ordered split-K reduction of
+//   gemm.cuh, and writes fp16 Y.
 //
-// Roles (12 warps): warp 0 lane 0 TMA producer; warp 1 lane 0 MMA issuer;
-// warps 2..7 unpack (nibbles to 16*q bytes, K-major, 128-byte swizzle, as in
-// gemm.cuh; the INT8 outlier group is copied) and lay the scales out; warps
-// 8..11 drain. Accumulators start at the conversion bias as in gemm.cuh.
+// A decode GEMM moves little data per SM (tens of KB) and does little work per
+// group, so what sets its time is how early the weights are requested and how
+// short each group's path is:
+//  * the packed ring has 8 slots, so the producer puts up to 8 groups of
+//    weights in flight at once (all of a K range of 8 groups at the start);
+//    each slot carries the group's packed W and A tiles and its sw by TMA, and
+//    its sa by 4-byte asynchronous copies from the producer warp's lanes (sa
+//    rows are M floats, which a TMA cannot address for M % 4 != 0; a register
+//    prefetch of them by plain loads made the producer wait on each group's
+//    loads and paced the whole kernel at ~0.6 us per group);
+//  * NT/16 drain warps per TMEM lane quarter, each with 16 token columns, so a
+//    group costs each drain warp one 16-column TMEM load;
+//  * four accumulators, so the MMA can run up to three groups ahead of the drain.
+//
+// Roles: warp 0 producer (lane 0 issues the tensor copies, all lanes the sa copies);
+// warp 1 lane 0 MMA issuer; warps 2..7 unpack (nibbles to 16*q bytes, K-major,
+// 128-byte swizzle, as in gemm.cuh; the INT8 outlier group is copied) and lay
+// the scales out; warps 8.. drain. Accumulators start at the conversion bias as
+// in gemm.cuh.
 #pragma once
 
 #include "gemm.cuh"
@@ -34,19 +47,26 @@ namespace atomk {
 namespace small_cfg {
 constexpr int BW = 128;                 // weight rows (output columns) per CTA
 constexpr int kMaxTokens = 64;          // token rows per call
-constexpr int kThreads = 384;
 constexpr int kUnpackThreads = 192;     // warps 2..7
 constexpr int kUnpackWarps = kUnpackThreads / 32;
-constexpr int kDrainWarps = 4;          // warps 8..11
-constexpr int kNP = 4, kNU = 3, kNS = 6;
-// packed slot: INT4 W (128 x 64 B) at 0 and INT4 A (64 x 64 B) at kPackAOff;
-// the INT8 group takes two slots: W8 (128 x 128 B), then A8 (64 x 128 B)
-constexpr uint32_t kPackAOff = BW * 64;
-constexpr uint32_t kPSlot = 17 * 1024;
+constexpr int kFirstDrainWarp = 8;
+constexpr int kNP = 8;                  // packed slots (groups of weights in flight)
+constexpr int kNU = 3;                  // operand slots
+constexpr int kNS = 8;                  // scale slots
+constexpr int kNB = 4;                  // TMEM accumulators, kMaxTokens columns apart
+// packed slot (1024-byte aligned). INT4 group: W4 (128 rows x 64 B) at 0, A4
+// (64 x 64 B) at kPackAOff. The INT8 group takes two slots; slot h holds W8
+// rows [64h, 64h+64) (64 x 128 B, 128-byte swizzle) at 0 and A8 rows
+// [32h, 32h+32) (32 x 128 B, swizzled) at kPackAOff. A group's first slot also
+// holds its sw (128 floats, by TMA) and sa (64 floats, by the producer's copies).
+constexpr uint32_t kPackAOff = 8192;
+constexpr uint32_t kPackSwOff = 12288;
+constexpr uint32_t kPackSaOff = kPackSwOff + BW * 4;
+constexpr uint32_t kPSlot = 13 * 1024;
 // operand slot: int8 W (128 x 128 B) then int8 A (64 x 128 B), K-major, 128-byte swizzle
 constexpr uint32_t kOpAOff = BW * 128;
 constexpr uint32_t kUSlot = kOpAOff + kMaxTokens * 128;
-// scale slot: per token pair (sa'[2j], sa'[2j+1], nc[2j], nc[2j+1]), then sw by weight row
+// scale slot: per token pair (sa'[2j], sa'[2j+1], -C*sa'[2j], -C*sa'[2j+1]), then sw by weight row
 constexpr uint32_t kSwOff = kMaxTokens * 8;
 constexpr uint32_t kSSlot = kSwOff + BW * 4;
 constexpr uint32_t kBarBytes = 1024;
@@ -54,20 +74,27 @@ constexpr uint32_t kPOff = kBarBytes;
 constexpr uint32_t kUOff = kPOff + kNP * kPSlot;
 constexpr uint32_t kSOff = kUOff + kNU * kUSlot;
 constexpr uint32_t kSmemBytes = kSOff + kNS * kSSlot + 1024;   // + alignment slack
-constexpr uint32_t kTmemCols = 2 * kMaxTokens;
+constexpr uint32_t kTmemCols = kNB * kMaxTokens;
+constexpr uint32_t kInt4Bytes = BW * 64 + kMaxTokens * 64 + BW * 4;   // TMA bytes of an INT4 slot
+constexpr uint32_t kInt8Bytes0 = 64 * 128 + 32 * 128 + BW * 4;       // first INT8 slot
+constexpr uint32_t kInt8Bytes1 = 64 * 128 + 32 * 128;                // second INT8 slot
 constexpr int kPackedChunks = (BW + kMaxTokens) * 4;            // 16-byte chunks, INT4 group
 constexpr int kInt8Chunks = (BW + kMaxTokens) * 8;              // 16-byte chunks, INT8 group
+__host__ __device__ constexpr int threads_for(int NT) { return 32 * (kFirstDrainWarp + NT / 4); }
 static_assert(kPSlot % 1024 == 0 && kUSlot % 1024 == 0 && kOpAOff % 1024 == 0, "1024-byte slots");
-static_assert(kPackAOff + kMaxTokens * 64 <= kPSlot && BW * 128 <= kPSlot, "packed slot");
+static_assert(kPackAOff + kMaxTokens * 64 <= kPackSwOff && kPackSaOff + kMaxTokens * 4 <= kPSlot,
+              "packed slot");
 static_assert(kPackedChunks % kUnpackThreads == 0 && kInt8Chunks % kUnpackThreads == 0, "chunks");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kTmemCols == 256, "TMEM allocation is a power of two");
 }  // namespace small_cfg
 
 struct SmallMaps {
   CUtensorMap w4;   // packed INT4 W: uint8 [N][(K-128)/2], boxes of 128 rows x 64 bytes
   CUtensorMap a4;   // packed INT4 A: uint8 [M][(K-128)/2], boxes of 64 rows x 64 bytes
-  CUtensorMap w8;   // INT8 W: [N][128], boxes 128 x 128 bytes, 128-byte swizzle
-  CUtensorMap a8;   // INT8 A: [M][128], boxes 64 x 128 bytes, 128-byte swizzle
+  CUtensorMap w8;   // INT8 W: [N][128], boxes 64 x 128 bytes, 128-byte swizzle
+  CUtensorMap a8;   // INT8 A: [M][128], boxes 32 x 128 bytes, 128-byte swizzle
+  CUtensorMap sw;   // fp32 [G][N], boxes of 1 x 128
 };
 
 struct SmallParams {
@@ -75,6 +102,7 @@ struct SmallParams {
   const float *sw;   // [G][N]
   __half *y;         // may be null in partials mode
   int32_t *partials; // partials mode only: int32 [G][M][N]
+  const uint8_t *qw4t;  // packed INT4 W in the tiled layout (tiled.cuh), or null: row layout by TMA
   int M, N, K, G;
   int n_tiles, splits, items;   // splits > 1: one item per CTA, a cluster of `splits` CTAs per tile
 };
@@ -117,23 +145,24 @@ __device__ __forceinline__ int64_t small_iterations(const SmallParams &p) {
 // arithmetic: P = (bits - bias) >> 8 for an INT4 group (the tiles hold 16*q, so
 // the MMA sums 256*P), bits - bias for the INT8 group.
 template <int NT, bool kPartials = false>
-__global__ void __launch_bounds__(small_cfg::kThreads, 1)
+__global__ void __launch_bounds__(small_cfg::threads_for(NT), 1)
 w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams p) {
   using namespace small_cfg;
   static_assert(NT == 16 || NT == 32 || NT == 64, "token tile");
   constexpr uint32_t kIdescSmall = idesc_i8(BW, NT);
+  constexpr int kDrainWarps = NT / 4;   // NT/16 per TMEM lane quarter
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
 
-  uint64_t *pfull = reinterpret_cast<uint64_t *>(smem);   // [kNP] TMA -> unpackers
+  uint64_t *pfull = reinterpret_cast<uint64_t *>(smem);   // [kNP] TMA + sa -> unpackers
   uint64_t *pempty = pfull + kNP;                         // [kNP] unpackers -> producer
   uint64_t *ufull = pempty + kNP;                         // [kNU] operands ready -> MMA
   uint64_t *uempty = ufull + kNU;                         // [kNU] MMA commit -> unpackers
   uint64_t *sfull = uempty + kNU;                         // [kNS] scales ready -> drain
   uint64_t *sempty = sfull + kNS;                         // [kNS] drain -> unpackers
-  uint64_t *tfull = sempty + kNS;                         // [2] accumulator complete
-  uint64_t *tempty = tfull + 2;                           // [2] accumulator drained
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  uint64_t *tfull = sempty + kNS;                         // [kNB] accumulator complete
+  uint64_t *tempty = tfull + kNB;                         // [kNB] accumulator drained
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + kNB);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   uint8_t *pring = smem + kPOff;
   uint8_t *uring = smem + kUOff;
@@ -142,7 +171,7 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNP; ++s) {
-      mbar_init(&pfull[s], 1);
+      mbar_init(&pfull[s], 33);  // 32 lanes' sa-copy arrivals + the expect_tx arrival
       mbar_init(&pempty[s], kUnpackWarps);
     }
     for (int s = 0; s < kNU; ++s) {
@@ -153,7 +182,7 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
       mbar_init(&sfull[s], kUnpackWarps);
       mbar_init(&sempty[s], kDrainWarps);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNB; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], kDrainWarps);
     }
@@ -170,13 +199,15 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
   const uint32_t tbase = *tmem_slot;
   const int64_t iters = small_iterations(p);
 
-  // both accumulators start at the conversion bias (see gemm.cuh)
-  if (warp >= 8) {
-    const uint32_t lanes = tbase + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+  // every accumulator starts at the conversion bias (see gemm.cuh): each drain
+  // warp fills its own 16 columns of each
+  if (warp >= kFirstDrainWarp) {
+    const int s = (warp - kFirstDrainWarp) >> 2;
+    const uint32_t lanes = tbase + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + 16 * s;
 #pragma unroll
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < kNB; ++b)
 #pragma unroll
-      for (int c = 0; c < NT / 4; ++c) tmem_st_x4_fill(lanes + b * kMaxTokens + 4 * c, gemm_cfg::kBias);
+      for (int c = 0; c < 4; ++c) tmem_st_x4_fill(lanes + b * kMaxTokens + 4 * c, gemm_cfg::kBias);
     tmem_st_wait();
   }
   tc_fence_before_sync();
@@ -188,25 +219,26 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
     *abort_flag = 1;
   };
 
-  if (warp >= 8) {
+  if (warp >= kFirstDrainWarp) {
     // ================================================================ drain
-    // Warp 8 + q owns TMEM lanes [32q, 32q+32): thread `lane` holds weight row
-    // n0 + 32q + lane and the NT token columns of its accumulator.
-    const int q = warp - 8;
+    // Warp 8 + 4s + q owns TMEM lanes [32q, 32q+32) and token columns
+    // [16s, 16s+16): thread `lane` holds weight row n0 + 32q + lane and the
+    // accumulators of those 16 tokens.
+    const int dw = warp - kFirstDrainWarp;
+    const int q = dw & 3, s = dw >> 2;
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
     const int lrow = 32 * q + lane;
-    float2 acc[NT / 2];
+    float2 acc[8];
 #pragma unroll
-    for (int i = 0; i < NT / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+    for (int i = 0; i < 8; ++i) acc[i] = make_float2(0.f, 0.f);
     SmallWalk w;
     w.start(p);
-    RingPos sr;
-    for (int64_t it = 0; it < iters; ++it, w.next(p), sr.next(kNS)) {
-      const int b = static_cast<int>(it & 1), sl = sr.idx;
-      const uint32_t tph = static_cast<uint32_t>((it >> 1) & 1);
-      bool ok = mbar_try_wait(&tfull[b], tph) & mbar_try_wait(&sfull[sl], sr.phase);
+    RingPos sr, br;
+    for (int64_t it = 0; it < iters; ++it, w.next(p), sr.next(kNS), br.next(kNB)) {
+      const int b = br.idx, sl = sr.idx;
+      bool ok = mbar_try_wait(&tfull[b], br.phase) & mbar_try_wait(&sfull[sl], sr.phase);
       if (!ok)
-        ok = mbar_wait(&tfull[b], tph, abort_flag) && mbar_wait(&sfull[sl], sr.phase, abort_flag);
+        ok = mbar_wait(&tfull[b], br.phase, abort_flag) && mbar_wait(&sfull[sl], sr.phase, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) fail();
         break;
@@ -214,42 +246,34 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
       tc_fence_after_sync();
       const uint8_t *ss = sring + sl * kSSlot;
       // per token pair: (sa'[2j], sa'[2j+1], -C*sa'[2j], -C*sa'[2j+1]); sa' as in gemm.cuh
-      const float4 *sap = reinterpret_cast<const float4 *>(ss);
+      const float4 *sap = reinterpret_cast<const float4 *>(ss) + 8 * s;
       const float swr = reinterpret_cast<const float *>(ss + kSwOff)[lrow];
       const float2 sw2 = make_float2(swr, swr);
-      const uint32_t tcol = tbase + lane_base + b * kMaxTokens;
-      uint32_t ra[16], rb[16];
-      tmem_ld_x16(tcol, ra);
-      tmem_ld_wait(ra);
+      const uint32_t tcol = tbase + lane_base + b * kMaxTokens + 16 * s;
+      uint32_t r[16];
+      tmem_ld_x16(tcol, r);
+      tmem_ld_wait(r);
+      if (kPartials) {
+        // weight row n, tokens 16s .. 16s+15; consecutive lanes write
+        // consecutive n of one token row
+        const int n = w.n0 + lrow;
+        const int sh = w.g < p.G - 1 ? 8 : 0;
 #pragma unroll
-      for (int c = 0; c < NT / 16; ++c) {
-        uint32_t(&r)[16] = (c & 1) ? rb : ra;
-        uint32_t(&rn)[16] = (c & 1) ? ra : rb;
-        if (c + 1 < NT / 16) tmem_ld_x16(tcol + 16 * (c + 1), rn);
-        if (kPartials) {
-          // weight row n, tokens 16c .. 16c+15; consecutive lanes write
-          // consecutive n of one token row
-          const int n = w.n0 + lrow;
-          const int sh = w.g < p.G - 1 ? 8 : 0;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int m = 16 * c + e;
-            if (n < p.N && m < p.M)
-              p.partials[(static_cast<int64_t>(w.g) * p.M + m) * p.N + n] =
-                  static_cast<int32_t>(r[e] - gemm_cfg::kBias) >> sh;
-          }
+        for (int e = 0; e < 16; ++e) {
+          const int m = 16 * s + e;
+          if (n < p.N && m < p.M)
+            p.partials[(static_cast<int64_t>(w.g) * p.M + m) * p.N + n] =
+                static_cast<int32_t>(r[e] - gemm_cfg::kBias) >> sh;
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {   // token pair 8c + j: columns 16c + 2j, 16c + 2j + 1
-          const float4 s4 = sap[8 * c + j];
-          const float2 f = make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-          float2 &a = acc[8 * c + j];
-          a = f2_fma(f2_fma(f, make_float2(s4.x, s4.y), make_float2(s4.z, s4.w)), sw2, a);
-        }
-        if (c + 1 < NT / 16) tmem_ld_wait(rn);
       }
 #pragma unroll
-      for (int e = 0; e < NT / 4; ++e) tmem_st_x4_fill(tcol + 4 * e, gemm_cfg::kBias);
+      for (int j = 0; j < 8; ++j) {   // token pair 8s + j: tokens 16s + 2j, 16s + 2j + 1
+        const float4 s4 = sap[j];
+        const float2 f = make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+        acc[j] = f2_fma(f2_fma(f, make_float2(s4.x, s4.y), make_float2(s4.z, s4.w)), sw2, acc[j]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) tmem_st_x4_fill(tcol + 4 * e, gemm_cfg::kBias);
       tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
@@ -267,10 +291,10 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
         const bool row_ok = n < p.N;
         float *part = reinterpret_cast<float *>(uring);
 #pragma unroll
-        for (int j = 0; j < NT / 2; ++j) {
+        for (int j = 0; j < 8; ++j) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int m = 2 * j + h;
+            const int m = 16 * s + 2 * j + h;
             const float v = h ? acc[j].y : acc[j].x;
             if (p.splits > 1)
               part[m * BW + lrow] = v;
@@ -283,54 +307,68 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
     }
   } else if (warp == 0) {
     // ================================================================ producer
-    if (lane == 0) {
-      SmallWalk wp;
-      wp.start(p);
-      RingPos pr;
-      int64_t ls = 0;
-      bool ok = true;
-      for (int64_t it = 0; ok && it < iters; ++it, wp.next(p)) {
-        const bool int4_group = wp.g < p.G - 1;
-        for (int part = 0; part < (int4_group ? 1 : 2); ++part) {
-          const int s = pr.idx;
-          if (!mbar_wait(&pempty[s], pr.phase ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t *slot = pring + s * kPSlot;
-          if (int4_group) {
-            mbar_arrive_expect_tx(&pfull[s], BW * 64u + kMaxTokens * 64u);
-            tma_load_2d(slot, &maps.w4, wp.g * 64, wp.n0, &pfull[s]);
-            tma_load_2d(slot + kPackAOff, &maps.a4, wp.g * 64, 0, &pfull[s]);
-          } else if (part == 0) {
-            mbar_arrive_expect_tx(&pfull[s], BW * 128u);
-            tma_load_2d(slot, &maps.w8, 0, wp.n0, &pfull[s]);
-          } else {
-            mbar_arrive_expect_tx(&pfull[s], kMaxTokens * 128u);
-            tma_load_2d(slot, &maps.a8, 0, 0, &pfull[s]);
-          }
-          ++ls;
-          pr.next(kNP);
+    // Lane 0 issues the tensor copies. Every lane copies sa for tokens
+    // 2*lane, 2*lane + 1 of the group into the group's first slot with 4-byte
+    // asynchronous copies, and arrives on the slot's barrier when they land
+    // (the barrier counts 32 such arrivals and lane 0's expect-tx arrival).
+    SmallWalk wp;
+    wp.start(p);
+    RingPos pr;
+    int64_t ls = 0;
+    bool ok = true;   // uniform across the warp (every wait is voted)
+    for (int64_t it = 0; ok && it < iters; ++it, wp.next(p)) {
+      const bool int4_group = wp.g < p.G - 1;
+      for (int part = 0; ok && part < (int4_group ? 1 : 2); ++part) {
+        const int s = pr.idx;
+        ok = __all_sync(0xffffffffu, mbar_wait(&pempty[s], pr.phase ^ 1u, abort_flag));
+        if (!ok) break;
+        uint8_t *slot = pring + s * kPSlot;
+        if (part == 0) {
+          const float *src = p.sa + static_cast<int64_t>(wp.g) * p.M;
+          const uint32_t dst = smem_addr(slot + kPackSaOff) + 8u * lane;
+          if (2 * lane < p.M) cp_async_4(dst, src + 2 * lane);
+          if (2 * lane + 1 < p.M) cp_async_4(dst + 4u, src + 2 * lane + 1);
         }
+        cp_async_mbar_arrive_noinc(&pfull[s]);
+        if (lane == 0) {
+          if (int4_group) {
+            mbar_arrive_expect_tx(&pfull[s], kInt4Bytes);
+            if (p.qw4t != nullptr)   // the tile's 8 KB block of the tiled layout
+              bulk_load(slot, p.qw4t + (static_cast<int64_t>(wp.n0 / BW) * (p.G - 1) + wp.g) *
+                                           (BW * 64),
+                        BW * 64u, &pfull[s]);
+            else
+              tma_load_2d(slot, &maps.w4, wp.g * 64, wp.n0, &pfull[s]);
+            tma_load_2d(slot + kPackAOff, &maps.a4, wp.g * 64, 0, &pfull[s]);
+          } else {
+            mbar_arrive_expect_tx(&pfull[s], part == 0 ? kInt8Bytes0 : kInt8Bytes1);
+            tma_load_2d(slot, &maps.w8, 0, wp.n0 + 64 * part, &pfull[s]);
+            tma_load_2d(slot + kPackAOff, &maps.a8, 0, 32 * part, &pfull[s]);
+          }
+          if (part == 0) tma_load_2d(slot + kPackSwOff, &maps.sw, wp.n0, wp.g, &pfull[s]);
+        }
+        ++ls;
+        pr.next(kNP);
       }
-      if (!ok) {
-        fail();
-        for (int64_t j = (ls > kNP ? ls - kNP : 0); j < ls; ++j)
-          (void)mbar_wait(&pfull[j % kNP], static_cast<uint32_t>((j / kNP) & 1), nullptr);
-      }
+    }
+    if (!ok && lane == 0) {
+      fail();
+      for (int64_t j = (ls > kNP ? ls - kNP : 0); j < ls; ++j)
+        (void)mbar_wait(&pfull[j % kNP], static_cast<uint32_t>((j / kNP) & 1), nullptr);
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
     if (lane == 0) {
       int64_t last_mma = -1;
+      int last_b = 0;
+      uint32_t last_ph = 0;
       bool ok = true;
-      RingPos ur;
-      for (int64_t it = 0; ok && it < iters; ++it, ur.next(kNU)) {
-        const int u = ur.idx, b = static_cast<int>(it & 1);
-        const uint32_t eph = static_cast<uint32_t>(((it >> 1) & 1) ^ 1);
-        if (!(mbar_try_wait(&ufull[u], ur.phase) & mbar_try_wait(&tempty[b], eph)) &&
+      RingPos ur, br;
+      for (int64_t it = 0; ok && it < iters; ++it, ur.next(kNU), br.next(kNB)) {
+        const int u = ur.idx, b = br.idx;
+        if (!(mbar_try_wait(&ufull[u], ur.phase) & mbar_try_wait(&tempty[b], br.phase ^ 1u)) &&
             (!mbar_wait(&ufull[u], ur.phase, abort_flag) ||
-             !mbar_wait(&tempty[b], eph, abort_flag))) {
+             !mbar_wait(&tempty[b], br.phase ^ 1u, abort_flag))) {
           ok = false;
           break;
         }
@@ -344,43 +382,20 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
         tc_commit(&tfull[b]);
         tc_commit(&uempty[u]);
         last_mma = it;
+        last_b = b;
+        last_ph = br.phase;
       }
       if (!ok) fail();
       // nothing may still write TMEM when it is released
-      if (last_mma >= 0)
-        (void)mbar_wait(&tfull[last_mma & 1], static_cast<uint32_t>((last_mma >> 1) & 1), nullptr);
+      if (last_mma >= 0) (void)mbar_wait(&tfull[last_b], last_ph, nullptr);
     }
   } else {
     // ================================================================ unpackers
     const int lt = threadIdx.x - 64;
-    // This thread's raw scales of a group: sw of weight row n0 + lt (lt < 128),
-    // or sa of tokens 2j, 2j+1 (j = lt - 128 < 32). They are fetched one group
-    // ahead, so that their global-memory latency is not on the group's path.
-    auto load_scales = [&](const SmallWalk &g, float (&v)[2]) {
-      v[0] = v[1] = 0.f;
-      if (lt < BW) {
-        const int n = g.n0 + lt;
-        if (n < p.N) v[0] = __ldg(p.sw + static_cast<int64_t>(g.g) * p.N + n);
-      } else if (lt < BW + kMaxTokens / 2) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int m = 2 * (lt - BW) + h;
-          if (m < p.M) v[h] = __ldg(p.sa + static_cast<int64_t>(g.g) * p.M + m);
-        }
-      }
-    };
     SmallWalk w;
     w.start(p);
-    float sc[2];
-    if (iters > 0) load_scales(w, sc);
     RingPos ur, sr, pr;
     for (int64_t it = 0; it < iters; ++it, ur.next(kNU), sr.next(kNS), w.next(p)) {
-      float sc_next[2] = {0.f, 0.f};
-      if (it + 1 < iters) {
-        SmallWalk w1 = w;
-        w1.next(p);
-        load_scales(w1, sc_next);
-      }
       const int u = ur.idx, sl = sr.idx;
       const bool int4_group = w.g < p.G - 1;
       const RingPos p0 = pr;
@@ -418,15 +433,21 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
           *reinterpret_cast<uint4 *>(dst + (((2 * cc + 1) ^ swz) << 4)) = hi;
         }
       } else {
-        // the INT8 group arrived already swizzled: W8 in slot p0, A8 in slot p1
+        // the INT8 group arrived already swizzled, in halves: slot p0 holds W8
+        // rows 0..63 and A8 rows 0..31, slot p1 the rest. 64 and 32 rows are
+        // whole 1024-byte swizzle atoms, so the halves are copied byte for byte.
         const uint8_t *pk1 = pring + p1.idx * kPSlot;
 #pragma unroll
         for (int i = 0; i < kInt8Chunks / kUnpackThreads; ++i) {
           const int c = lt + kUnpackThreads * i;
           const bool is_w = c < BW * 8;
-          const uint32_t off = (is_w ? c : c - BW * 8) * 16u;
-          *reinterpret_cast<uint4 *>(op + (is_w ? 0u : kOpAOff) + off) =
-              *reinterpret_cast<const uint4 *>((is_w ? pk : pk1) + off);
+          const int cw = is_w ? c : c - BW * 8;               // chunk within W8 (1024) or A8 (512)
+          const int half_chunks = is_w ? BW * 4 : kMaxTokens * 4;
+          const int h = cw >= half_chunks;
+          const uint32_t off = (cw - h * half_chunks) * 16u;
+          const uint8_t *src = (h ? pk1 : pk) + (is_w ? 0u : kPackAOff) + off;
+          uint8_t *dst = op + (is_w ? 0u : kOpAOff) + h * half_chunks * 16u + off;
+          *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
         }
       }
       // scales: sw of the tile's weight rows, and per token pair
@@ -435,15 +456,17 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
       // fp32 steps as gemm.cuh's drain
       uint8_t *ss = sring + sl * kSSlot;
       if (lt < BW) {
-        reinterpret_cast<float *>(ss + kSwOff)[lt] = sc[0];
+        reinterpret_cast<float *>(ss + kSwOff)[lt] =
+            reinterpret_cast<const float *>(pk + kPackSwOff)[lt];
       } else if (lt < BW + kMaxTokens / 2) {
         const int j = lt - BW;
-        float sv[2];
+        const float2 sa = reinterpret_cast<const float2 *>(pk + kPackSaOff)[j];
+        float sv[2] = {sa.x, sa.y};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          float s = sc[h];
-          if (int4_group) s *= 0.00390625f;
-          sv[h] = __uint_as_float(__float_as_uint(s) & 0xFFFFFFFCu);
+          float v = sv[h];
+          if (int4_group) v *= 0.00390625f;
+          sv[h] = __uint_as_float(__float_as_uint(v) & 0xFFFFFFFCu);
         }
         reinterpret_cast<float4 *>(ss)[j] =
             make_float4(sv[0], sv[1], -gemm_cfg::kBiasF * sv[0], -gemm_cfg::kBiasF * sv[1]);
@@ -458,8 +481,6 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
       }
       pr = p1;
       if (!int4_group) pr.next(kNP);
-      sc[0] = sc_next[0];
-      sc[1] = sc_next[1];
     }
   }
 
@@ -478,7 +499,7 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
     const int n0 = (static_cast<int>(blockIdx.x) / S) * BW;
     const int lo = rank * BW / S, nr = (rank + 1) * BW / S - lo;
     const float *part = reinterpret_cast<const float *>(uring);
-    for (int e = threadIdx.x; e < p.M * nr; e += kThreads) {
+    for (int e = threadIdx.x; e < p.M * nr; e += threads_for(NT)) {
       const int m = e / nr, row = lo + (e - m * nr);
       const float *src = part + m * BW + row;
       float v = ld_shared_cluster_f32(cluster_map(src, 0));

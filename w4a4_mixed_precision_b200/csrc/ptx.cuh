@@ -143,6 +143,20 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void 
                : "memory");
 }
 
+// 4-byte asynchronous copy global -> shared (no register is written, so no
+// later instruction waits on it); completion is tracked per thread.
+__device__ __forceinline__ void cp_async_4(uint32_t dst_smem, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+
+// Arrives on `bar` (without raising its expected count: the barrier's count
+// must include this arrival) once every cp.async this thread issued so far
+// has completed.
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -163,6 +177,10 @@ __device__ __forceinline__ void st_shared_v4(void *dst, uint32_t a, uint32_t b, 
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(dst)), "r"(a), "r"(b),
                "r"(c), "r"(d)
                : "memory");
+}
+
+__device__ __forceinline__ void st_shared_b32(void *dst, uint32_t a) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(smem_addr(dst)), "r"(a) : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05
@@ -410,6 +428,38 @@ __device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, ui
       "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// 2-SM MMA of fp16 operands with an fp32 accumulator: D (+)= A * B^T.
+__device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Instruction descriptor for kind::f16: f32 accumulator, f16 x f16, K-major A and B.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+  return (1u << 4)                                   // D format: f32
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Shared-memory matrix descriptor for a K-major tile without swizzle: core
+// matrices of 8 rows x 16 bytes (128 contiguous bytes); `lbo` is the byte
+// distance between core matrices adjacent in K, `sbo` between core matrices
+// adjacent in M/N.
+__device__ __forceinline__ uint64_t smem_desc_k_noswizzle(uint32_t saddr, uint32_t lbo,
+                                                          uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // start address
+  d |= static_cast<uint64_t>(lbo >> 4) << 16;           // leading (K) byte offset
+  d |= static_cast<uint64_t>(sbo >> 4) << 32;           // stride (M/N) byte offset
+  d |= static_cast<uint64_t>(1) << 46;                  // descriptor version (sm_100)
+  return d;                                             // swizzle mode 0: none
 }
 
 // Arrives on the barrier at this shared-memory offset in every CTA of
