@@ -42,6 +42,11 @@
  *    if the caller is checking a different stream's work;
  *  - the fixed scratch array of atom_w4a4_gemm_noalloc: calls of that entry
  *    point that overlap on the GPU race on it and must be ordered by the caller.
+ *  - the quantizers' row counters (atom_reorder_quant, atom_quant_weights): a
+ *    ring of 1024 per device, handed out one per call in call order and reset
+ *    by the launch that used it. Quantizer launches whose call numbers on the
+ *    device differ by a multiple of 1024 must not run at the same time (that
+ *    takes 1024 or more quantizer launches in flight at once).
  * Apart from these, calls on different streams that share no output buffer and
  * no workspace may run concurrently.
  */

@@ -36,6 +36,7 @@ struct DeviceState {
   int w8a8_clusters = 0;          // co-resident CTA pairs of the W8A8 kernel
   uint32_t quant_smem_set = 0;
   std::atomic<void *> noalloc_scratch{nullptr};  // device address of g_noalloc_scratch here
+  std::atomic<uint32_t> quant_calls{0};   // picks each quantizer call's row-counter slot
 };
 
 DeviceState g_devices[kMaxDevices];
@@ -113,10 +114,15 @@ atom_status_t launch_quant(const void *x, int64_t rows, int64_t K, int64_t ld,
     }
   }
   const int grid = static_cast<int>(rows < dev->sm_count ? rows : dev->sm_count);
+  // The launch's row counter: slots go round in call order, so launches that
+  // run at the same time use different slots unless kQuantSlots or more
+  // quantizer calls of this device are in flight at once.
+  const int slot = static_cast<int>(dev->quant_calls.fetch_add(1, std::memory_order_relaxed) %
+                                    static_cast<uint32_t>(atomk::kQuantSlots));
   atomk::reorder_quant_kernel<<<grid, atomk::kQuantThreads, L.total,
                                 reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const __half *>(x), rows, static_cast<int>(K), ld, idx, q4, q8, scales,
-      static_cast<int>(stages), static_cast<int>(crews), a8 ? 1 : 0);
+      static_cast<int>(stages), static_cast<int>(crews), a8 ? 1 : 0, slot);
   return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
 }
 
@@ -141,21 +147,72 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps, by their encoding arguments. A map depends only on the
+// address, sizes, strides, box and swizzle it is built from (not on the data
+// or on the device's state), so an identical request can reuse it; serving
+// loops call the same GEMM on the same buffers again and again, and encoding
+// the five to seven maps of a call on the host costs more than a decode GEMM
+// takes on the GPU. Direct-mapped, guarded by g_map_mutex.
+struct MapKey {
+  const void *base;
+  uint64_t cols, rows, stride;
+  uint32_t box_cols, box_rows;
+  int dtype, swizzle;
+  bool operator==(const MapKey &o) const {
+    return base == o.base && cols == o.cols && rows == o.rows && stride == o.stride &&
+           box_cols == o.box_cols && box_rows == o.box_rows && dtype == o.dtype &&
+           swizzle == o.swizzle;
+  }
+};
+struct MapEntry {
+  bool valid = false;
+  MapKey key;
+  CUtensorMap map;
+};
+constexpr int kMapCacheSize = 256;
+MapEntry g_map_cache[kMapCacheSize];
+std::mutex g_map_mutex;
+
+size_t map_slot(const MapKey &k) {
+  uint64_t h = reinterpret_cast<uintptr_t>(k.base) * 0x9E3779B97F4A7C15ull;
+  for (uint64_t v : {k.cols, k.rows, k.stride, static_cast<uint64_t>(k.box_cols),
+                     static_cast<uint64_t>(k.box_rows), static_cast<uint64_t>(k.dtype),
+                     static_cast<uint64_t>(k.swizzle)})
+    h = (h ^ v) * 0x100000001B3ull;
+  return static_cast<size_t>(h >> 32) % kMapCacheSize;
+}
+
 // 2-D tensor map over a row-major matrix of `rows` rows, `cols` elements per
 // row and a row stride of `stride_bytes`, copied in boxes of box_rows x box_cols;
 // reads past the matrix edge fill with zeros.
 bool encode_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, uint64_t cols,
                uint64_t rows, uint64_t stride_bytes, uint32_t box_cols, uint32_t box_rows,
                CUtensorMapSwizzle swizzle) {
+  const MapKey key{base, cols, rows, stride_bytes, box_cols, box_rows, static_cast<int>(dtype),
+                   static_cast<int>(swizzle)};
+  const size_t slot = map_slot(key);
+  {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    if (g_map_cache[slot].valid && g_map_cache[slot].key == key) {
+      *map = g_map_cache[slot].map;
+      return true;
+    }
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {stride_bytes};
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::lock_guard<std::mutex> lock(g_map_mutex);
+  g_map_cache[slot].key = key;
+  g_map_cache[slot].map = *map;
+  g_map_cache[slot].valid = true;
+  return true;
 }
 
 // K splits for a GEMM whose output tiles would leave most CTA pairs idle

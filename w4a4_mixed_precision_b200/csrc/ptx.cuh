@@ -179,10 +179,6 @@ __device__ __forceinline__ void st_shared_v4(void *dst, uint32_t a, uint32_t b, 
                : "memory");
 }
 
-__device__ __forceinline__ void st_shared_b32(void *dst, uint32_t a) {
-  asm volatile("st.shared.b32 [%0], %1;" ::"r"(smem_addr(dst)), "r"(a) : "memory");
-}
-
 // ------------------------------------------------------------------ tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {

@@ -9,16 +9,21 @@
 //
 // Design (HBM-bound, so the aim is to keep HBM busy with few instructions per
 // element):
-//  * one CTA per SM, persistent over rows r = blockIdx.x + i*gridDim.x. It
-//    runs up to three crews, each of 8 quantizing warps and one copy-issuing
-//    warp with its own ring of 2-4 stage slots: the copy warp takes the CTA's
-//    next row from a counter in shared memory whenever a slot of its ring is
-//    free, tags the slot with the row, and brings the whole fp16 row in with
-//    one bulk copy (TMA engine, mbarrier completion); each quantizing warp
-//    frees a slot through its own arrival on an "empty" mbarrier. A crew the
-//    warp scheduler favours thus takes more rows, and the crews end together;
-//    run as three separate CTAs per SM, with fixed rows each, the last one
-//    ended ~25 % after the first;
+//  * one CTA per SM, persistent. It runs up to three crews, each of 8
+//    quantizing warps and one copy-issuing warp with its own ring of 2-4 stage
+//    slots: the copy warp takes the next row of the whole launch from a row
+//    counter in global memory whenever a slot of its ring is free, tags the
+//    slot with the row, and brings the whole fp16 row in with one bulk copy
+//    (TMA engine, mbarrier completion); each quantizing warp frees a slot
+//    through its own arrival on an "empty" mbarrier. A crew or an SM that runs
+//    faster thus takes more rows, and all end together: with fixed rows per
+//    SM, the same few SMs ended each launch 10-15 us (a quarter of a launch)
+//    after the rest. The copy warp keeps one row claimed ahead, so the
+//    counter's round trip is off the refill path;
+//  * the row counter is one of kQuantSlots slots that the host hands out in
+//    turn, one per call; the last CTA of a launch to finish puts its slot back
+//    to zero, so the slot is ready for its next call, or for the next replay
+//    of a captured launch;
 //  * at start-up each CTA (once per SM, shared by its crews) turns the outlier
 //    list into a gather table in shared
 //    memory (uint16 [K]): for every group and lane, the byte offsets inside a
@@ -28,7 +33,9 @@
 //    block scan of the non-outlier counts);
 //  * 8 lanes quantize one group (16 elements per lane), 4 groups per warp per
 //    pass: two conflict-free 16-byte table loads, 16 gathered halves, amax by
-//    shuffles over the 8 lanes, one IEEE division each for scale and inv, code
+//    shuffles over the 8 lanes; scale and inv of an INT4 group from a
+//    1024-entry table of IEEE quotients by the significand of amax (see
+//    kDivTable), of the INT8 group by one IEEE division each; code
 //    bits from the low byte of fp32(1.5*2^23 + x*inv) (round half to even,
 //    exact for |t| < 2^22), byte permutes to
 //    pack, one 8-byte (INT4) or 16-byte (INT8) store per lane;
@@ -50,18 +57,33 @@ constexpr int kQuantMaxStages = 12;
 constexpr uint32_t kQHdrFull = 0;                            // uint64 [kQuantMaxStages]
 constexpr uint32_t kQHdrEmpty = kQHdrFull + 8 * kQuantMaxStages;
 constexpr uint32_t kQHdrFlags = kQHdrEmpty + 8 * kQuantMaxStages;  // int [2]: bad list, abort
-constexpr uint32_t kQHdrNext = kQHdrFlags + 8;               // int: next row to claim
-constexpr uint32_t kQHdrTags = kQHdrNext + 8;                // int [kQuantMaxStages]: row of each slot
-constexpr uint32_t kQHdrSums = 256;                          // int [32]: block-scan partials
+constexpr uint32_t kQHdrTags = kQHdrFlags + 8;               // int64 [kQuantMaxStages]: row of each slot
+constexpr uint32_t kQHdrSums = 320;                          // int [32]: block-scan partials
 constexpr uint32_t kQHdrBytes = kQHdrSums + 4 * 32;
-static_assert(kQHdrTags + 4 * kQuantMaxStages <= kQHdrSums, "quantizer header");
+static_assert(kQHdrTags + 8 * kQuantMaxStages <= kQHdrSums, "quantizer header");
 static_assert(kQuantThreads <= 1024, "quantizer block");
 // Gather-table entries are 16-bit byte offsets into a staged fp16 row.
 constexpr int kQuantMaxK = 32768;
 
+// Row counters shared by the launches of one device: a launch claims rows
+// from g_quant_next[slot] and counts its finished CTAs in g_quant_exits[slot];
+// the last one resets both. Zero at module load.
+constexpr int kQuantSlots = 1024;
+__device__ unsigned long long g_quant_next[kQuantSlots];
+__device__ unsigned int g_quant_exits[kQuantSlots];
+
+// Scale and inverse scale of an INT4 group, by the significand of its
+// maximum. The maximum is an fp16 value, so its fp32 significand has at most
+// 10 fraction bits: 1 + f/1024 for f < 1024, times a power of two 2^E. Entry f
+// holds RN((1 + f/1024)/7) and RN(7/(1 + f/1024)), each one IEEE division;
+// the group's RN(amax/7) and RN(7/amax) are those entries times 2^E and 2^-E
+// (a power of two scales a correctly rounded quotient exactly while it stays a
+// normal number, and for fp16 inputs both always do: from 2^-27 to 2^26).
+constexpr int kDivTable = 1024;
+
 struct QuantLayout {
   // Byte offsets inside dynamic shared memory.
-  uint32_t bitmap, wbase, table, stages, total;
+  uint32_t bitmap, wbase, table, divtab, stages, total;
   uint32_t row_bytes;
   int stages_n;
 };
@@ -72,7 +94,8 @@ __host__ __device__ inline QuantLayout quant_layout(int K, int stages_n) {
   L.bitmap = kQHdrBytes;                                           // after the header
   L.wbase = L.bitmap + ((static_cast<uint32_t>(K) / 8u + 15u) & ~15u);   // int [K/32]
   L.table = L.wbase + ((static_cast<uint32_t>(K) / 8u + 15u) & ~15u);
-  L.stages = (L.table + L.row_bytes + 127u) & ~127u;
+  L.divtab = (L.table + L.row_bytes + 15u) & ~15u;                 // float2 [kDivTable]
+  L.stages = (L.divtab + 8u * kDivTable + 127u) & ~127u;
   L.stages_n = stages_n;
   L.total = L.stages + static_cast<uint32_t>(stages_n) * L.row_bytes;
   return L;
@@ -97,31 +120,29 @@ __device__ __forceinline__ int quant_table_index(int p, int Gd, bool a8) {
 }
 
 
-__global__ void __launch_bounds__(kQuantThreads, 1)
-reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t ld,
-                     const int32_t *__restrict__ outlier_idx, uint8_t *__restrict__ q4,
-                     int8_t *__restrict__ q8, float *__restrict__ scales, int stages_n,
-                     int crews_n, int a8) {
-  extern __shared__ __align__(1024) uint8_t smem[];
+// The work of one CTA; every thread returns from here to the launch-end
+// bookkeeping of reorder_quant_kernel.
+__device__ __forceinline__ void
+reorder_quant_cta(uint8_t *smem, const __half *__restrict__ x, int64_t rows, int K, int64_t ld,
+                  const int32_t *__restrict__ outlier_idx, uint8_t *__restrict__ q4,
+                  int8_t *__restrict__ q8, float *__restrict__ scales, int stages_n, int crews_n,
+                  int a8, unsigned long long *next) {
   const QuantLayout L = quant_layout(K, stages_n * crews_n);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kQHdrFull);
   uint64_t *empty = reinterpret_cast<uint64_t *>(smem + kQHdrEmpty);
   volatile int *flags = reinterpret_cast<volatile int *>(smem + kQHdrFlags);  // [0] bad list, [1] abort
-  int *next_row = reinterpret_cast<int *>(smem + kQHdrNext);
-  volatile int *tags = reinterpret_cast<volatile int *>(smem + kQHdrTags);
+  volatile int64_t *tags = reinterpret_cast<volatile int64_t *>(smem + kQHdrTags);
   int *warp_sums = reinterpret_cast<int *>(smem + kQHdrSums);
   uint32_t *bitmap = reinterpret_cast<uint32_t *>(smem + L.bitmap);
   int *wbase = reinterpret_cast<int *>(smem + L.wbase);
   uint16_t *table = reinterpret_cast<uint16_t *>(smem + L.table);
+  float2 *divtab = reinterpret_cast<float2 *>(smem + L.divtab);
   uint8_t *stage_base = smem + L.stages;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int crew = warp / (kQuantWarps + 1), cw = warp % (kQuantWarps + 1);
   const int G = K / 128, Gd = G - 1, Kd = K - 128;
   const int64_t q4_row = Kd / 2;
-  const int64_t grid = gridDim.x;
-  // this CTA's rows are blockIdx.x + i*grid for i < n_rows (grid <= rows)
-  const int64_t n_rows = (rows - blockIdx.x + grid - 1) / grid;
   // the outlier list is read once, as early as possible
   const int oc = tid < 128 ? __ldg(outlier_idx + tid) : 0;
 
@@ -132,31 +153,36 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
     }
     flags[0] = 0;
     flags[1] = 0;
-    *next_row = 0;
     fence_mbar_init();
   }
   for (int w = tid; w < K / 32; w += kQuantThreads) bitmap[w] = 0u;
+  for (int f = tid; f < kDivTable; f += kQuantThreads) {
+    const float m = __uint_as_float(0x3F800000u | (static_cast<uint32_t>(f) << 13));
+    divtab[f] = make_float2(__fdiv_rn(m, 7.f), __fdiv_rn(7.f, m));
+  }
   __syncthreads();
 
   // This crew's ring: stages_n slots with their barriers and row tags.
   uint64_t *cfull = full + crew * stages_n;
   uint64_t *cempty = empty + crew * stages_n;
-  volatile int *ctags = tags + crew * stages_n;
+  volatile int64_t *ctags = tags + crew * stages_n;
   uint8_t *cstage = stage_base + static_cast<size_t>(crew) * stages_n * L.row_bytes;
   const bool copier = cw == kQuantWarps && lane == 0 && crew < crews_n;
-  // Takes the CTA's next row for ring slot s and puts it in flight; past the
-  // last row it completes the slot's phase with a plain arrival and a tag
-  // >= n_rows instead, which tells the crew to stop.
+  // `ahead` is the row claimed ahead: claim() puts it in flight in ring slot
+  // s and takes the next one from the launch's counter; past the last row it
+  // completes the slot's phase with a plain arrival and a tag >= rows instead,
+  // which tells the crew to stop, and claims nothing more.
+  int64_t ahead = copier ? static_cast<int64_t>(atomicAdd(next, 1ull)) : rows;
   auto claim = [&](int s) -> bool {
-    const int i = atomicAdd(next_row, 1);
-    ctags[s] = i;
-    if (i >= n_rows) {
+    const int64_t r = ahead;
+    ctags[s] = r;
+    if (r >= rows) {
       mbar_arrive(&cfull[s]);
       return false;
     }
-    const int64_t r = blockIdx.x + static_cast<int64_t>(i) * grid;
     mbar_arrive_expect_tx(&cfull[s], L.row_bytes);
     bulk_load(cstage + s * L.row_bytes, x + r * ld, L.row_bytes, &cfull[s]);
+    ahead = static_cast<int64_t>(atomicAdd(next, 1ull));
     return true;
   };
   // Each crew's first row goes in flight before the table is built, the rest
@@ -290,9 +316,8 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
       }
       break;
     }
-    const int i = ctags[s];
-    if (i >= n_rows) break;
-    const int64_t r = blockIdx.x + static_cast<int64_t>(i) * grid;
+    const int64_t r = ctags[s];
+    if (r >= rows) break;
     const uint8_t *row = cstage + s * L.row_bytes;
     uint8_t *q4_r = q4 + r * q4_row;
     int8_t *q8_r = q8 + r * (a8 ? static_cast<int64_t>(K) : 128);
@@ -317,15 +342,25 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
       amax = fmaxf(amax, __shfl_xor_sync(team_mask, amax, 4));
       amax = fmaxf(amax, __shfl_xor_sync(team_mask, amax, 2));
       amax = fmaxf(amax, __shfl_xor_sync(team_mask, amax, 1));
-      const float qmax = dense ? 7.f : 127.f;
       float scale = 0.f, inv = 0.f;
-      if (amax > 0.f) {
-        scale = __fdiv_rn(amax, qmax);
-        inv = __fdiv_rn(qmax, amax);
+      if (dense) {
+        // amax = (1 + f/1024) * 2^E: entry f, exponent moved by E
+        const uint32_t ab = __float_as_uint(amax);
+        const float2 t = divtab[(ab >> 13) & (kDivTable - 1)];
+        const uint32_t e = (ab & 0x7F800000u) - 0x3F800000u;   // E << 23 (two's complement)
+        if (amax > 0.f) {
+          scale = __uint_as_float(__float_as_uint(t.x) + e);
+          inv = __uint_as_float(__float_as_uint(t.y) - e);
+        }
+      } else if (amax > 0.f) {
+        scale = __fdiv_rn(amax, 127.f);
+        inv = __fdiv_rn(127.f, amax);
       }
-      // code bits: the low byte of fp32(1.5*2^23 + rint(x*inv)) is the two's complement code
-      // __fmul_rn/__fadd_rn are never contracted into an FMA: the product must
-      // be rounded to fp32 before the 1.5*2^23 add rounds it to an integer.
+      // code bits: the low byte of fp32(1.5*2^23 + rint(x*inv)) is the two's
+      // complement code. The product is rounded to fp32 before the 1.5*2^23 add
+      // rounds it to an integer (separate instructions, never one FMA).
+      // (Scalar instructions: the packed f32x2 multiply and add were fused
+      // into one f32x2 FMA by the compiler, which skips the product's rounding.)
       uint32_t b[16];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -365,6 +400,26 @@ reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t 
       s = 0;
       ph ^= 1u;
     }
+  }
+}
+
+// One launch over all rows, its row counter in slot `slot`. Each CTA counts
+// itself out once its copy warps have made their last claim; the last one
+// resets the slot, when no claim of this launch can follow.
+__global__ void __launch_bounds__(kQuantThreads, 1)
+reorder_quant_kernel(const __half *__restrict__ x, int64_t rows, int K, int64_t ld,
+                     const int32_t *__restrict__ outlier_idx, uint8_t *__restrict__ q4,
+                     int8_t *__restrict__ q8, float *__restrict__ scales, int stages_n,
+                     int crews_n, int a8, int slot) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  reorder_quant_cta(smem, x, rows, K, ld, outlier_idx, q4, q8, scales, stages_n, crews_n, a8,
+                    g_quant_next + slot);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0 && atomicAdd(g_quant_exits + slot, 1u) == gridDim.x - 1) {
+    __threadfence();
+    g_quant_next[slot] = 0ull;
+    g_quant_exits[slot] = 0u;
   }
 }
 
