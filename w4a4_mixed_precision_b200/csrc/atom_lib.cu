@@ -241,7 +241,7 @@ atom_status_t gemm_pairs(DeviceState *dev, int mode, int *pairs);   // mode + 3 
 // CTA, as many K ranges (of at least 2 groups, at most 8: they form one
 // thread-block cluster of portable size) as keep every SM busy without a
 // second wave. 1 = no split.
-constexpr int kMaxSmallSplits = 8;
+constexpr int kMaxSmallSplits = atomk::small_cfg::kMaxSplits;
 int small_splits(int64_t N, int64_t K, int sms) {
   const int64_t n_tiles = (N + atomk::small_cfg::BW - 1) / atomk::small_cfg::BW;
   if (n_tiles <= 0 || n_tiles >= sms) return 1;

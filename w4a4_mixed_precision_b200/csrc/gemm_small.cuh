@@ -29,15 +29,21 @@
 //    rows are M floats, which a TMA cannot address for M % 4 != 0; a register
 //    prefetch of them by plain loads made the producer wait on each group's
 //    loads and paced the whole kernel at ~0.6 us per group);
+//  * the producer starts as soon as the barriers exist: the TMEM allocation
+//    runs beside the first loads;
 //  * NT/16 drain warps per TMEM lane quarter, each with 16 token columns, so a
-//    group costs each drain warp one 16-column TMEM load;
-//  * four accumulators, so the MMA can run up to three groups ahead of the drain.
+//    group costs each drain warp one 16-column TMEM load; an fp16 MMA of
+//    constant tiles starts each group's accumulator at the conversion bias (as
+//    in gemm.cuh), so the drain writes nothing back to TMEM;
+//  * four accumulators, so the MMA can run up to three groups ahead of the drain;
+//  * the split-K reduction issues all of an element's distributed-shared-memory
+//    loads before it adds them (in K-range order), four elements per thread at
+//    a time.
 //
-// Roles: warp 0 producer (lane 0 issues the tensor copies, all lanes the sa copies);
-// warp 1 lane 0 MMA issuer; warps 2..7 unpack (nibbles to 16*q bytes, K-major,
-// 128-byte swizzle, as in gemm.cuh; the INT8 outlier group is copied) and lay
-// the scales out; warps 8.. drain. Accumulators start at the conversion bias as
-// in gemm.cuh.
+// Roles: warp 0 producer (lane 0 issues the tensor copies, all lanes the sa
+// copies); warp 1 allocates TMEM, its lane 0 issues the MMAs; warps 2..7 unpack
+// (nibbles to 16*q bytes, K-major, 128-byte swizzle, as in gemm.cuh; the INT8
+// outlier group is copied) and lay the scales out; warps 8.. drain.
 #pragma once
 
 #include "gemm.cuh"
@@ -54,6 +60,7 @@ constexpr int kNP = 8;                  // packed slots (groups of weights in fl
 constexpr int kNU = 3;                  // operand slots
 constexpr int kNS = 8;                  // scale slots
 constexpr int kNB = 4;                  // TMEM accumulators, kMaxTokens columns apart
+constexpr int kMaxSplits = 8;           // most K ranges of a tile (a portable cluster)
 // packed slot (1024-byte aligned). INT4 group: W4 (128 rows x 64 B) at 0, A4
 // (64 x 64 B) at kPackAOff. The INT8 group takes two slots; slot h holds W8
 // rows [64h, 64h+64) (64 x 128 B, 128-byte swizzle) at 0 and A8 rows
@@ -73,7 +80,12 @@ constexpr uint32_t kBarBytes = 1024;
 constexpr uint32_t kPOff = kBarBytes;
 constexpr uint32_t kUOff = kPOff + kNP * kPSlot;
 constexpr uint32_t kSOff = kUOff + kNU * kUSlot;
-constexpr uint32_t kSmemBytes = kSOff + kNS * kSSlot + 1024;   // + alignment slack
+// bias tiles of the fp16 MMA: A (BW rows) then B (kMaxTokens rows), 16 fp16
+// per row, K-major without swizzle (core matrices of 8 rows x 16 bytes)
+constexpr uint32_t kBiasOff = kSOff + kNS * kSSlot;
+constexpr uint32_t kBiasA = BW * 32, kBiasB = kMaxTokens * 32;
+constexpr uint32_t kBiasLbo = 128, kBiasSbo = 256;
+constexpr uint32_t kSmemBytes = kBiasOff + kBiasA + kBiasB + 1024;   // + alignment slack
 constexpr uint32_t kTmemCols = kNB * kMaxTokens;
 constexpr uint32_t kInt4Bytes = BW * 64 + kMaxTokens * 64 + BW * 4;   // TMA bytes of an INT4 slot
 constexpr uint32_t kInt8Bytes0 = 64 * 128 + 32 * 128 + BW * 4;       // first INT8 slot
@@ -150,6 +162,7 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
   using namespace small_cfg;
   static_assert(NT == 16 || NT == 32 || NT == 64, "token tile");
   constexpr uint32_t kIdescSmall = idesc_i8(BW, NT);
+  constexpr uint32_t kIdescBias = idesc_f16(BW, NT);
   constexpr int kDrainWarps = NT / 4;   // NT/16 per TMEM lane quarter
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -189,30 +202,29 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+  // the bias tiles: element (row, k = 0) = 6144 (A) or 2048 (B), all else 0
+  for (int i = threadIdx.x; i < static_cast<int>((kBiasA + kBiasB) / 16); i += threads_for(NT)) {
+    const int t = i >= static_cast<int>(kBiasA / 16), j = (i >> 3) & 1;
+    const uint32_t v = j == 0 ? (t == 0 ? 0x6E00u : 0x6800u) : 0u;   // fp16 6144 / 2048
+    reinterpret_cast<uint4 *>(smem + kBiasOff)[i] = make_uint4(v, 0u, 0u, 0u);
   }
-  tc_fence_before_sync();
+  fence_proxy_async_smem();
   __syncthreads();
-  tc_fence_after_sync();
-  const uint32_t tbase = *tmem_slot;
   const int64_t iters = small_iterations(p);
 
-  // every accumulator starts at the conversion bias (see gemm.cuh): each drain
-  // warp fills its own 16 columns of each
-  if (warp >= kFirstDrainWarp) {
-    const int s = (warp - kFirstDrainWarp) >> 2;
-    const uint32_t lanes = tbase + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + 16 * s;
-#pragma unroll
-    for (int b = 0; b < kNB; ++b)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_st_x4_fill(lanes + b * kMaxTokens + 4 * c, gemm_cfg::kBias);
-    tmem_st_wait();
+  // TMEM: allocated by warp 1 while the producer already loads; warp 1 and the
+  // drain warps meet at named barrier 1 to learn its address
+  uint32_t tbase = 0;
+  if (warp == 1 || warp >= kFirstDrainWarp) {
+    if (warp == 1) {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish();
+      tc_fence_before_sync();
+    }
+    named_bar_sync(1, 32 * (1 + kDrainWarps));
+    tc_fence_after_sync();
+    tbase = *tmem_slot;
   }
-  tc_fence_before_sync();
-  __syncthreads();
-  tc_fence_after_sync();
 
   auto fail = [&](void) {
     report_status(6 /* ATOM_ERR_TIMEOUT */);
@@ -272,9 +284,6 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
         const float2 f = make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
         acc[j] = f2_fma(f2_fma(f, make_float2(s4.x, s4.y), make_float2(s4.z, s4.w)), sw2, acc[j]);
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) tmem_st_x4_fill(tcol + 4 * e, gemm_cfg::kBias);
-      tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) {
@@ -364,6 +373,10 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
       uint32_t last_ph = 0;
       bool ok = true;
       RingPos ur, br;
+      const uint64_t bias_adesc =
+          smem_desc_k_noswizzle(smem_addr(smem + kBiasOff), kBiasLbo, kBiasSbo);
+      const uint64_t bias_bdesc =
+          smem_desc_k_noswizzle(smem_addr(smem + kBiasOff + kBiasA), kBiasLbo, kBiasSbo);
       for (int64_t it = 0; ok && it < iters; ++it, ur.next(kNU), br.next(kNB)) {
         const int u = ur.idx, b = br.idx;
         if (!(mbar_try_wait(&ufull[u], ur.phase) & mbar_try_wait(&tempty[b], br.phase ^ 1u)) &&
@@ -377,6 +390,8 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
         const uint64_t adesc = smem_desc_k_sw128(op);             // weights, 128 rows
         const uint64_t bdesc = smem_desc_k_sw128(op + kOpAOff);   // tokens, NT rows
         const uint32_t d = tbase + b * kMaxTokens;
+        // the accumulator starts at the conversion bias (fp16 MMA of the constant tiles)
+        mma_f16(d, bias_adesc, bias_bdesc, kIdescBias, 0u);
 #pragma unroll
         for (int k = 0; k < 4; ++k) mma_i8(d, adesc + 2 * k, bdesc + 2 * k, kIdescSmall, 1u);
         tc_commit(&tfull[b]);
@@ -486,7 +501,7 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
 
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after_sync();
     tmem_dealloc(tbase, kTmemCols);
   }
@@ -499,12 +514,33 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
     const int n0 = (static_cast<int>(blockIdx.x) / S) * BW;
     const int lo = rank * BW / S, nr = (rank + 1) * BW / S - lo;
     const float *part = reinterpret_cast<const float *>(uring);
-    for (int e = threadIdx.x; e < p.M * nr; e += threads_for(NT)) {
-      const int m = e / nr, row = lo + (e - m * nr);
-      const float *src = part + m * BW + row;
-      float v = ld_shared_cluster_f32(cluster_map(src, 0));
-      for (int r = 1; r < S; ++r) v += ld_shared_cluster_f32(cluster_map(src, r));
-      if (n0 + row < p.N) p.y[static_cast<int64_t>(m) * p.N + n0 + row] = __float2half_rn(v);
+    constexpr int kE = 4;                 // elements per thread in flight
+    const int total = p.M * nr;
+    for (int e0 = threadIdx.x; e0 < total; e0 += kE * threads_for(NT)) {
+      float v[kE][kMaxSplits];
+#pragma unroll
+      for (int u = 0; u < kE; ++u) {
+        const int e = e0 + u * threads_for(NT);
+        if (e < total) {
+          const int m = e / nr, row = lo + (e - m * nr);
+          const float *src = part + m * BW + row;
+#pragma unroll
+          for (int r = 0; r < kMaxSplits; ++r)
+            if (r < S) v[u][r] = ld_shared_cluster_f32(cluster_map(src, r));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kE; ++u) {
+        const int e = e0 + u * threads_for(NT);
+        if (e < total) {
+          const int m = e / nr, row = lo + (e - m * nr);
+          float acc = v[u][0];
+#pragma unroll
+          for (int r = 1; r < kMaxSplits; ++r)
+            if (r < S) acc += v[u][r];
+          if (n0 + row < p.N) p.y[static_cast<int64_t>(m) * p.N + n0 + row] = __float2half_rn(acc);
+        }
+      }
     }
     cluster_sync();   // no CTA leaves while a peer may still read its tile
   }
