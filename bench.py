@@ -198,6 +198,30 @@ def _time_cycle(fns, n, stream):
     return e0.elapsed_time(e1) / n
 
 
+def _time_graph(fns, n, stream):
+    """Average ms per call of the same round-robin sequence of n calls, captured
+    once in a CUDA graph on `stream` and replayed (one untimed replay first):
+    the device time of the calls without the host's per-call launch cost."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            fns[i % len(fns)]()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):   # replay() launches on the current stream
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    del g
+    return ms
+
+
 def _copies_for(bytes_per_set: float, cap: int = 16) -> int:
     """Input sets to rotate through so that consecutive calls never find their
     operands in the 126 MB L2 (at least two sets, and more than twice L2)."""
@@ -258,23 +282,29 @@ def per_config_legs(configs, dev, stream, n_calls, int8_peak, int8_probe, hbm_gb
         ys = [torch.empty((w.M, w.N), dtype=torch.float16, device=dev) for _ in range(n_sets)]
         wss = [atom.gemm_workspace(w.M, w.N, w.K, dev) for _ in range(n_sets)]
 
-        def gemm_fn(i):
-            return lambda: atom.atom_w4a4_gemm(qas[i], qws[i], w.K, y=ys[i], stream=stream,
+        gs = torch.cuda.Stream()   # graph capture needs a stream other than the default one
+
+        def gemm_fn(i, st):
+            return lambda: atom.atom_w4a4_gemm(qas[i], qws[i], w.K, y=ys[i], stream=st,
                                                workspace=wss[i])
-        g_ms = _time_cycle([gemm_fn(i) for i in range(n_sets)], n_calls, stream)
+        g_ms = _time_cycle([gemm_fn(i, stream) for i in range(n_sets)], n_calls, stream)
+        g_ms_graph = _time_graph([gemm_fn(i, gs) for i in range(n_sets)], n_calls, gs)
         n_qsets = _copies_for(quant_bytes)
         As = [A] + [A.clone() for _ in range(n_qsets - 1)]
         qouts = [atom.empty_quantized(w.M, w.K, dev) for _ in range(n_qsets)]
 
-        def quant_fn(i):
-            return lambda: atom.atom_reorder_quant(As[i], idx, out=qouts[i], stream=stream)
-        q_ms = _time_cycle([quant_fn(i) for i in range(n_qsets)], n_calls, stream)
+        def quant_fn(i, st):
+            return lambda: atom.atom_reorder_quant(As[i], idx, out=qouts[i], stream=st)
+        q_ms = _time_cycle([quant_fn(i, stream) for i in range(n_qsets)], n_calls, stream)
+        q_ms_graph = _time_graph([quant_fn(i, gs) for i in range(n_qsets)], n_calls, gs)
         del As, qouts, qas, ys, wss
         n_csets = _copies_for(2.0 * (w.M + w.N) * w.K + 2.0 * w.M * w.N)
         Ws = [W16] + [W16.clone() for _ in range(n_csets - 1)]
         yc = torch.empty((w.M, w.N), dtype=torch.float16, device=dev)
-        c_ms = _time_cycle([(lambda Wi: (lambda: torch.matmul(A, Wi.t(), out=yc)))(Wi)
-                            for Wi in Ws], n_calls, stream)
+        c_fns = [(lambda Wi: (lambda: torch.matmul(A, Wi.t(), out=yc)))(Wi) for Wi in Ws]
+        c_ms = _time_cycle(c_fns, n_calls, stream)
+        with torch.cuda.stream(gs):
+            c_ms_graph = _time_graph(c_fns, n_calls, gs)
         del Ws, yc, W16, A
         if atom.atom_device_status(clear=True) != 0:
             raise RuntimeError(f"device status set on workload {c}")
@@ -282,6 +312,8 @@ def per_config_legs(configs, dev, stream, n_calls, int8_peak, int8_probe, hbm_gb
         entry = {
             "workload": f"{w.name} M={w.M} N={w.N} K={w.K}",
             "gemm_us": round(g_ms * 1e3, 2),
+            "gemm_us_graph": round(g_ms_graph * 1e3, 2),
+            "gemm_gbs_graph": round(gemm_bytes / (g_ms_graph * 1e-3) / 1e9, 1),
             "gemm_tops": round(g_tops, 2),
             "gemm_frac_int8_peak": round(g_tops / int8_peak, 4),
             "gemm_frac_int8_probe": round(g_tops / int8_probe, 4) if int8_probe else None,
@@ -290,13 +322,18 @@ def per_config_legs(configs, dev, stream, n_calls, int8_peak, int8_probe, hbm_gb
             "gemm_frac_hbm": round(gemm_bytes / (g_ms * 1e-3) / 1e9 / hbm_gbs, 4),
             "gemm_splits_workspace_bytes": atom.atom_gemm_workspace_bytes(w.M, w.N, w.K),
             "quant_us": round(q_ms * 1e3, 2),
+            "quant_us_graph": round(q_ms_graph * 1e3, 2),
             "quant_bytes": quant_bytes,
             "quant_gbs": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
             "quant_frac_hbm": round(quant_bytes / (q_ms * 1e-3) / 1e9 / hbm_gbs, 4),
             "fp16_cublas_us": round(c_ms * 1e3, 2),
+            "fp16_cublas_us_graph": round(c_ms_graph * 1e3, 2),
             "fp16_cublas_tflops": round(ops / (c_ms * 1e-3) / 1e12, 2),
             "w4a4_gemm_speedup_vs_fp16": round(c_ms / g_ms, 3),
             "calls": n_calls,
+            "timing": "*_us: CUDA events around `calls` calls issued back to back from Python "
+                      "(host launch cost included); *_us_graph: the same calls captured in one "
+                      "CUDA graph and replayed (device time per call)",
             "l2": f"GEMM rotates {n_sets} input sets, quantizer {n_qsets}, cuBLAS {n_csets} "
                   f"weight copies (each rotation more than twice the 126 MB L2, or 16 sets)",
             "bound": "hbm" if c == 1 else "tensor",
