@@ -610,6 +610,8 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
         const int row0 = w.m0 + BM * rank + 32 * q;   // the warp's first row
         float *ws_row = p.ws + (static_cast<int64_t>(w.split) * p.M + (row < p.M ? row : 0)) * p.N;
         uint8_t *ybuf = ystage + dw * kYSlot;
+        // Y is written once and not read here: first out of L2
+        const uint64_t y_policy = l2_policy_evict_first();
 #pragma unroll
         for (int v = 0; v < 16; ++v) {
           if ((v & 7) == 0) {
@@ -630,7 +632,7 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
             __syncwarp();
             const int col0 = w.n0 + kHalfN * hh + 64 * (v >> 3);
             if (lane == 0 && to_y && row0 < p.M && col0 < p.N) {
-              tma_store_2d(&maps.y, ybuf, col0, row0);
+              tma_store_2d_hint(&maps.y, ybuf, col0, row0, y_policy);
               bulk_commit_group();
             }
           }
@@ -646,6 +648,9 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     if (warp == 0) {
       // ============================================================== producer
       if (lane == 0) {
+        // A's tiles are read again for every column of output tiles: keep
+        // them in L2 ahead of the streaming Y writes
+        const uint64_t a_policy = l2_policy_evict_last();
         TileWalk wp;
         wp.start(p);
         int64_t ls = 0;   // packed-ring load steps issued
@@ -683,11 +688,11 @@ w4a4_gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
                                      (p.sa_by_tma ? BM * 4u : 0u);
               mbar_arrive_expect_tx(&pfull[s], bytes);
               if (!two_slots) {
-                tma_load_2d(slot, &maps.a4, wp.g * 64, arow, &pfull[s]);
+                tma_load_2d_hint(slot, &maps.a4, wp.g * 64, arow, &pfull[s], a_policy);
                 load_w4(slot + kPackWOff);
               } else {
                 // W4A4: the INT8 outlier tile of A ([M][128]); W4A8: group g of A ([M][K])
-                tma_load_2d(slot, &maps.a8, kA8 ? wp.g * 128 : 0, arow, &pfull[s]);
+                tma_load_2d_hint(slot, &maps.a8, kA8 ? wp.g * 128 : 0, arow, &pfull[s], a_policy);
               }
               tma_load_2d(slot + kSwLinOff, &maps.sw, wp.n0, wp.g, &pfull[s]);
               if (p.sa_by_tma) tma_load_2d(slot + kSaLinOff, &maps.sa, arow, wp.g, &pfull[s]);

@@ -120,6 +120,31 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
       : "memory");
 }
 
+// L2 eviction-priority policies for the cache-hinted copies below: data read
+// again soon (evict_last), and data written once and not read back here
+// (evict_first).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// tma_load_2d with an L2 eviction-priority policy for the lines it brings in.
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *map, int32_t x,
+                                                 int32_t y, uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
 // 2-D tiled tensor copy global -> shared (no multicast). x is the innermost
 // coordinate and must be 16-byte aligned in bytes.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int32_t x,
@@ -141,6 +166,16 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void 
                    reinterpret_cast<uint64_t>(map)),
                "r"(x), "r"(y), "r"(smem_addr(src))
                : "memory");
+}
+
+// tma_store_2d with an L2 eviction-priority policy for the lines it writes.
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap *map, const void *src,
+                                                  int32_t x, int32_t y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;" ::
+          "l"(reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(smem_addr(src)), "l"(policy)
+      : "memory");
 }
 
 // 4-byte asynchronous copy global -> shared (no register is written, so no
