@@ -57,10 +57,15 @@ constexpr int kUnpackThreads = 192;     // warps 2..7
 constexpr int kUnpackWarps = kUnpackThreads / 32;
 constexpr int kFirstDrainWarp = 8;
 constexpr int kNP = 8;                  // packed slots (groups of weights in flight)
-constexpr int kNU = 3;                  // operand slots
+constexpr int kNU = 4;                  // operand slots (one group each)
 constexpr int kNS = 8;                  // scale slots
 constexpr int kNB = 4;                  // TMEM accumulators, kMaxTokens columns apart
 constexpr int kMaxSplits = 8;           // most K ranges of a tile (a portable cluster)
+// The unpack, MMA and drain roles advance in steps of two INT4 groups (one
+// when a K range has an odd INT4 group left, and the INT8 group alone): each
+// step takes a pair of operand slots, a pair of scale slots and a pair of
+// accumulators, with one barrier per pair.
+constexpr int kUS = kNU / 2, kSS = kNS / 2, kBS = kNB / 2;
 // packed slot (1024-byte aligned). INT4 group: W4 (128 rows x 64 B) at 0, A4
 // (64 x 64 B) at kPackAOff. The INT8 group takes two slots; slot h holds W8
 // rows [64h, 64h+64) (64 x 128 B, 128-byte swizzle) at 0 and A8 rows
@@ -152,6 +157,36 @@ __device__ __forceinline__ int64_t small_iterations(const SmallParams &p) {
   return n;
 }
 
+// The step sequence of the unpack, MMA and drain roles: w at a step's first
+// group, n groups in it (2 when the next group is an INT4 group of the same K
+// range, else 1).
+struct SmallStep {
+  SmallWalk w;
+  int n;
+  __device__ __forceinline__ void fix(const SmallParams &p) {
+    n = (w.g + 1 < w.g_end && w.g + 1 < p.G - 1) ? 2 : 1;
+  }
+  __device__ __forceinline__ void start(const SmallParams &p) {
+    w.start(p);
+    fix(p);
+  }
+  __device__ __forceinline__ bool last() const { return w.g + n == w.g_end; }
+  __device__ __forceinline__ void next(const SmallParams &p) {
+    for (int i = 0; i < n; ++i) w.next(p);
+    fix(p);
+  }
+};
+
+__device__ __forceinline__ int64_t small_steps(const SmallParams &p) {
+  int64_t n = 0;
+  for (int it = blockIdx.x; it < p.items; it += gridDim.x) {
+    const int s = it % p.splits;
+    const int g1 = (s + 1) * p.G / p.splits;
+    for (int g = s * p.G / p.splits; g < g1; ++n) g += (g + 1 < g1 && g + 1 < p.G - 1) ? 2 : 1;
+  }
+  return n;
+}
+
 // kPartials: also write each group's exact int32 partial sums P[g][m][n] (the
 // debug entry point), read from the biased accumulator before the scale
 // arithmetic: P = (bits - bias) >> 8 for an INT4 group (the tiles hold 16*q, so
@@ -169,13 +204,13 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
 
   uint64_t *pfull = reinterpret_cast<uint64_t *>(smem);   // [kNP] TMA + sa -> unpackers
   uint64_t *pempty = pfull + kNP;                         // [kNP] unpackers -> producer
-  uint64_t *ufull = pempty + kNP;                         // [kNU] operands ready -> MMA
-  uint64_t *uempty = ufull + kNU;                         // [kNU] MMA commit -> unpackers
-  uint64_t *sfull = uempty + kNU;                         // [kNS] scales ready -> drain
-  uint64_t *sempty = sfull + kNS;                         // [kNS] drain -> unpackers
-  uint64_t *tfull = sempty + kNS;                         // [kNB] accumulator complete
-  uint64_t *tempty = tfull + kNB;                         // [kNB] accumulator drained
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + kNB);
+  uint64_t *ufull = pempty + kNP;                         // [kUS] operand pair ready -> MMA
+  uint64_t *uempty = ufull + kUS;                         // [kUS] MMA commit -> unpackers
+  uint64_t *sfull = uempty + kUS;                         // [kSS] scale pair ready -> drain
+  uint64_t *sempty = sfull + kSS;                         // [kSS] drain -> unpackers
+  uint64_t *tfull = sempty + kSS;                         // [kBS] accumulator pair complete
+  uint64_t *tempty = tfull + kBS;                         // [kBS] accumulator pair drained
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + kBS);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   uint8_t *pring = smem + kPOff;
   uint8_t *uring = smem + kUOff;
@@ -187,15 +222,15 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
       mbar_init(&pfull[s], 33);  // 32 lanes' sa-copy arrivals + the expect_tx arrival
       mbar_init(&pempty[s], kUnpackWarps);
     }
-    for (int s = 0; s < kNU; ++s) {
+    for (int s = 0; s < kUS; ++s) {
       mbar_init(&ufull[s], kUnpackWarps);
       mbar_init(&uempty[s], 1);
     }
-    for (int s = 0; s < kNS; ++s) {
+    for (int s = 0; s < kSS; ++s) {
       mbar_init(&sfull[s], kUnpackWarps);
       mbar_init(&sempty[s], kDrainWarps);
     }
-    for (int i = 0; i < kNB; ++i) {
+    for (int i = 0; i < kBS; ++i) {
       mbar_init(&tfull[i], 1);
       mbar_init(&tempty[i], kDrainWarps);
     }
@@ -210,7 +245,8 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
   }
   fence_proxy_async_smem();
   __syncthreads();
-  const int64_t iters = small_iterations(p);
+  const int64_t iters = small_iterations(p);   // groups (producer)
+  const int64_t steps = small_steps(p);        // steps (unpack, MMA, drain)
 
   // TMEM: allocated by warp 1 while the producer already loads; warp 1 and the
   // drain warps meet at named barrier 1 to learn its address
@@ -243,10 +279,10 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
     float2 acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = make_float2(0.f, 0.f);
-    SmallWalk w;
-    w.start(p);
+    SmallStep st;
+    st.start(p);
     RingPos sr, br;
-    for (int64_t it = 0; it < iters; ++it, w.next(p), sr.next(kNS), br.next(kNB)) {
+    for (int64_t it = 0; it < steps; ++it, st.next(p), sr.next(kSS), br.next(kBS)) {
       const int b = br.idx, sl = sr.idx;
       bool ok = mbar_try_wait(&tfull[b], br.phase) & mbar_try_wait(&sfull[sl], sr.phase);
       if (!ok)
@@ -256,33 +292,37 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
         break;
       }
       tc_fence_after_sync();
-      const uint8_t *ss = sring + sl * kSSlot;
-      // per token pair: (sa'[2j], sa'[2j+1], -C*sa'[2j], -C*sa'[2j+1]); sa' as in gemm.cuh
-      const float4 *sap = reinterpret_cast<const float4 *>(ss) + 8 * s;
-      const float swr = reinterpret_cast<const float *>(ss + kSwOff)[lrow];
-      const float2 sw2 = make_float2(swr, swr);
-      const uint32_t tcol = tbase + lane_base + b * kMaxTokens + 16 * s;
-      uint32_t r[16];
-      tmem_ld_x16(tcol, r);
-      tmem_ld_wait(r);
-      if (kPartials) {
-        // weight row n, tokens 16s .. 16s+15; consecutive lanes write
-        // consecutive n of one token row
-        const int n = w.n0 + lrow;
-        const int sh = w.g < p.G - 1 ? 8 : 0;
+      // the step's groups in order: accumulator 2b + j, scale slot 2sl + j
+      for (int j = 0; j < st.n; ++j) {
+        const int g = st.w.g + j;
+        const uint8_t *ss = sring + (2 * sl + j) * kSSlot;
+        // per token pair: (sa'[2j], sa'[2j+1], -C*sa'[2j], -C*sa'[2j+1]); sa' as in gemm.cuh
+        const float4 *sap = reinterpret_cast<const float4 *>(ss) + 8 * s;
+        const float swr = reinterpret_cast<const float *>(ss + kSwOff)[lrow];
+        const float2 sw2 = make_float2(swr, swr);
+        const uint32_t tcol = tbase + lane_base + (2 * b + j) * kMaxTokens + 16 * s;
+        uint32_t r[16];
+        tmem_ld_x16(tcol, r);
+        tmem_ld_wait(r);
+        if (kPartials) {
+          // weight row n, tokens 16s .. 16s+15; consecutive lanes write
+          // consecutive n of one token row
+          const int n = st.w.n0 + lrow;
+          const int sh = g < p.G - 1 ? 8 : 0;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int m = 16 * s + e;
-          if (n < p.N && m < p.M)
-            p.partials[(static_cast<int64_t>(w.g) * p.M + m) * p.N + n] =
-                static_cast<int32_t>(r[e] - gemm_cfg::kBias) >> sh;
+          for (int e = 0; e < 16; ++e) {
+            const int m = 16 * s + e;
+            if (n < p.N && m < p.M)
+              p.partials[(static_cast<int64_t>(g) * p.M + m) * p.N + n] =
+                  static_cast<int32_t>(r[e] - gemm_cfg::kBias) >> sh;
+          }
         }
-      }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {   // token pair 8s + j: tokens 16s + 2j, 16s + 2j + 1
-        const float4 s4 = sap[j];
-        const float2 f = make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-        acc[j] = f2_fma(f2_fma(f, make_float2(s4.x, s4.y), make_float2(s4.z, s4.w)), sw2, acc[j]);
+        for (int k = 0; k < 8; ++k) {   // token pair 8s + k: tokens 16s + 2k, 16s + 2k + 1
+          const float4 s4 = sap[k];
+          const float2 f = make_float2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+          acc[k] = f2_fma(f2_fma(f, make_float2(s4.x, s4.y), make_float2(s4.z, s4.w)), sw2, acc[k]);
+        }
       }
       tc_fence_before_sync();
       __syncwarp();
@@ -290,27 +330,27 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
         mbar_arrive(&tempty[b]);
         mbar_arrive(&sempty[sl]);
       }
-      if (w.last()) {
+      if (st.last()) {
         // this K range of the item is complete: write the thread's row of Y
         // (tokens m < M); with a split, park the range's fp32 partial tile
         // [token][weight row] in the operand ring, which no MMA reads any more
         // (the item is the CTA's only one). Consecutive lanes take consecutive
         // columns.
-        const int n = w.n0 + lrow;
+        const int n = st.w.n0 + lrow;
         const bool row_ok = n < p.N;
         float *part = reinterpret_cast<float *>(uring);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int k = 0; k < 8; ++k) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int m = 16 * s + 2 * j + h;
-            const float v = h ? acc[j].y : acc[j].x;
+            const int m = 16 * s + 2 * k + h;
+            const float v = h ? acc[k].y : acc[k].x;
             if (p.splits > 1)
               part[m * BW + lrow] = v;
             else if (row_ok && m < p.M && p.y != nullptr)
               p.y[static_cast<int64_t>(m) * p.N + n] = __float2half_rn(v);
           }
-          acc[j] = make_float2(0.f, 0.f);
+          acc[k] = make_float2(0.f, 0.f);
         }
       }
     }
@@ -377,7 +417,9 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
           smem_desc_k_noswizzle(smem_addr(smem + kBiasOff), kBiasLbo, kBiasSbo);
       const uint64_t bias_bdesc =
           smem_desc_k_noswizzle(smem_addr(smem + kBiasOff + kBiasA), kBiasLbo, kBiasSbo);
-      for (int64_t it = 0; ok && it < iters; ++it, ur.next(kNU), br.next(kNB)) {
+      SmallStep st;
+      st.start(p);
+      for (int64_t it = 0; ok && it < steps; ++it, ur.next(kUS), br.next(kBS), st.next(p)) {
         const int u = ur.idx, b = br.idx;
         if (!(mbar_try_wait(&ufull[u], ur.phase) & mbar_try_wait(&tempty[b], br.phase ^ 1u)) &&
             (!mbar_wait(&ufull[u], ur.phase, abort_flag) ||
@@ -386,14 +428,16 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
           break;
         }
         tc_fence_after_sync();
-        const uint32_t op = smem_addr(uring + u * kUSlot);
-        const uint64_t adesc = smem_desc_k_sw128(op);             // weights, 128 rows
-        const uint64_t bdesc = smem_desc_k_sw128(op + kOpAOff);   // tokens, NT rows
-        const uint32_t d = tbase + b * kMaxTokens;
-        // the accumulator starts at the conversion bias (fp16 MMA of the constant tiles)
-        mma_f16(d, bias_adesc, bias_bdesc, kIdescBias, 0u);
+        for (int j = 0; j < st.n; ++j) {
+          const uint32_t op = smem_addr(uring + (2 * u + j) * kUSlot);
+          const uint64_t adesc = smem_desc_k_sw128(op);             // weights, 128 rows
+          const uint64_t bdesc = smem_desc_k_sw128(op + kOpAOff);   // tokens, NT rows
+          const uint32_t d = tbase + (2 * b + j) * kMaxTokens;
+          // the accumulator starts at the conversion bias (fp16 MMA of the constant tiles)
+          mma_f16(d, bias_adesc, bias_bdesc, kIdescBias, 0u);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) mma_i8(d, adesc + 2 * k, bdesc + 2 * k, kIdescSmall, 1u);
+          for (int k = 0; k < 4; ++k) mma_i8(d, adesc + 2 * k, bdesc + 2 * k, kIdescSmall, 1u);
+        }
         tc_commit(&tfull[b]);
         tc_commit(&uempty[u]);
         last_mma = it;
@@ -407,12 +451,14 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
   } else {
     // ================================================================ unpackers
     const int lt = threadIdx.x - 64;
-    SmallWalk w;
-    w.start(p);
+    SmallStep st;
+    st.start(p);
     RingPos ur, sr, pr;
-    for (int64_t it = 0; it < iters; ++it, ur.next(kNU), sr.next(kNS), w.next(p)) {
+    for (int64_t it = 0; it < steps; ++it, ur.next(kUS), sr.next(kSS), st.next(p)) {
       const int u = ur.idx, sl = sr.idx;
-      const bool int4_group = w.g < p.G - 1;
+      const int n = st.n;
+      const bool int4_step = st.w.g < p.G - 1;
+      const bool two = !int4_step || n == 2;   // the step takes two packed slots
       const RingPos p0 = pr;
       RingPos p1 = pr;
       p1.next(kNP);
@@ -422,36 +468,57 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
         ok = mbar_wait(&uempty[u], ur.phase ^ 1u, abort_flag) &&
              mbar_wait(&sempty[sl], sr.phase ^ 1u, abort_flag) &&
              mbar_wait(&pfull[p0.idx], p0.phase, abort_flag);
-      if (ok && !int4_group) ok = mbar_wait(&pfull[p1.idx], p1.phase, abort_flag);
+      if (ok && two) ok = mbar_wait(&pfull[p1.idx], p1.phase, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) fail();
         break;
       }
-      const uint8_t *pk = pring + p0.idx * kPSlot;
-      uint8_t *op = uring + u * kUSlot;
-      if (int4_group) {
-        // nibbles -> bytes holding 16*q, K-major with the 128-byte swizzle
+      const uint8_t *pk0 = pring + p0.idx * kPSlot, *pk1 = pring + p1.idx * kPSlot;
+      if (int4_step) {
+        // nibbles -> bytes holding 16*q, K-major with the 128-byte swizzle;
+        // group j of the step into operand slot 2u + j. Every shared-memory
+        // load of the step goes out before the first store.
+        constexpr int kCh = kPackedChunks / kUnpackThreads;
+        uint4 v[2][kCh];
 #pragma unroll
-        for (int i = 0; i < kPackedChunks / kUnpackThreads; ++i) {
-          const int c = lt + kUnpackThreads * i;
-          const bool is_w = c < BW * 4;
-          const int row = (is_w ? c : c - BW * 4) >> 2, cc = c & 3;
-          const uint4 v =
-              *reinterpret_cast<const uint4 *>(pk + (is_w ? 0u : kPackAOff) + row * 64 + cc * 16);
-          uint8_t *dst = op + (is_w ? 0u : kOpAOff) + row * 128;
-          const uint4 lo = make_uint4((v.x << 4) & 0xF0F0F0F0u, (v.y << 4) & 0xF0F0F0F0u,
-                                      (v.z << 4) & 0xF0F0F0F0u, (v.w << 4) & 0xF0F0F0F0u);
-          const uint4 hi = make_uint4(v.x & 0xF0F0F0F0u, v.y & 0xF0F0F0F0u, v.z & 0xF0F0F0F0u,
-                                      v.w & 0xF0F0F0F0u);
-          const int swz = row & 7;
-          *reinterpret_cast<uint4 *>(dst + (((2 * cc) ^ swz) << 4)) = lo;
-          *reinterpret_cast<uint4 *>(dst + (((2 * cc + 1) ^ swz) << 4)) = hi;
+        for (int j = 0; j < 2; ++j) {
+          if (j < n) {
+#pragma unroll
+            for (int i = 0; i < kCh; ++i) {
+              const int c = lt + kUnpackThreads * i;
+              const bool is_w = c < BW * 4;
+              const int row = (is_w ? c : c - BW * 4) >> 2, cc = c & 3;
+              v[j][i] = *reinterpret_cast<const uint4 *>((j ? pk1 : pk0) + (is_w ? 0u : kPackAOff) +
+                                                          row * 64 + cc * 16);
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (j < n) {
+            uint8_t *op = uring + (2 * u + j) * kUSlot;
+#pragma unroll
+            for (int i = 0; i < kCh; ++i) {
+              const int c = lt + kUnpackThreads * i;
+              const bool is_w = c < BW * 4;
+              const int row = (is_w ? c : c - BW * 4) >> 2, cc = c & 3;
+              const uint4 x = v[j][i];
+              uint8_t *dst = op + (is_w ? 0u : kOpAOff) + row * 128;
+              const uint4 lo = make_uint4((x.x << 4) & 0xF0F0F0F0u, (x.y << 4) & 0xF0F0F0F0u,
+                                          (x.z << 4) & 0xF0F0F0F0u, (x.w << 4) & 0xF0F0F0F0u);
+              const uint4 hi = make_uint4(x.x & 0xF0F0F0F0u, x.y & 0xF0F0F0F0u,
+                                          x.z & 0xF0F0F0F0u, x.w & 0xF0F0F0F0u);
+              const int swz = row & 7;
+              *reinterpret_cast<uint4 *>(dst + (((2 * cc) ^ swz) << 4)) = lo;
+              *reinterpret_cast<uint4 *>(dst + (((2 * cc + 1) ^ swz) << 4)) = hi;
+            }
+          }
         }
       } else {
         // the INT8 group arrived already swizzled, in halves: slot p0 holds W8
         // rows 0..63 and A8 rows 0..31, slot p1 the rest. 64 and 32 rows are
         // whole 1024-byte swizzle atoms, so the halves are copied byte for byte.
-        const uint8_t *pk1 = pring + p1.idx * kPSlot;
+        uint8_t *op = uring + 2 * u * kUSlot;
 #pragma unroll
         for (int i = 0; i < kInt8Chunks / kUnpackThreads; ++i) {
           const int c = lt + kUnpackThreads * i;
@@ -460,42 +527,45 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
           const int half_chunks = is_w ? BW * 4 : kMaxTokens * 4;
           const int h = cw >= half_chunks;
           const uint32_t off = (cw - h * half_chunks) * 16u;
-          const uint8_t *src = (h ? pk1 : pk) + (is_w ? 0u : kPackAOff) + off;
+          const uint8_t *src = (h ? pk1 : pk0) + (is_w ? 0u : kPackAOff) + off;
           uint8_t *dst = op + (is_w ? 0u : kOpAOff) + h * half_chunks * 16u + off;
           *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(src);
         }
       }
-      // scales: sw of the tile's weight rows, and per token pair
-      // (sa'[2j], sa'[2j+1], -C*sa'[2j], -C*sa'[2j+1]) with sa' = sa (times
-      // 1/256 for an INT4 group) truncated to 22 significant bits, the same
-      // fp32 steps as gemm.cuh's drain
-      uint8_t *ss = sring + sl * kSSlot;
-      if (lt < BW) {
-        reinterpret_cast<float *>(ss + kSwOff)[lt] =
-            reinterpret_cast<const float *>(pk + kPackSwOff)[lt];
-      } else if (lt < BW + kMaxTokens / 2) {
-        const int j = lt - BW;
-        const float2 sa = reinterpret_cast<const float2 *>(pk + kPackSaOff)[j];
-        float sv[2] = {sa.x, sa.y};
+      // scales of group j into scale slot 2sl + j: sw of the tile's weight
+      // rows, and per token pair (sa'[2k], sa'[2k+1], -C*sa'[2k],
+      // -C*sa'[2k+1]) with sa' = sa (times 1/256 for an INT4 group) truncated
+      // to 22 significant bits, the same fp32 steps as gemm.cuh's drain
+      for (int j = 0; j < n; ++j) {
+        const uint8_t *pk = j ? pk1 : pk0;
+        uint8_t *ss = sring + (2 * sl + j) * kSSlot;
+        if (lt < BW) {
+          reinterpret_cast<float *>(ss + kSwOff)[lt] =
+              reinterpret_cast<const float *>(pk + kPackSwOff)[lt];
+        } else if (lt < BW + kMaxTokens / 2) {
+          const int k = lt - BW;
+          const float2 sa = reinterpret_cast<const float2 *>(pk + kPackSaOff)[k];
+          float sv[2] = {sa.x, sa.y};
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float v = sv[h];
-          if (int4_group) v *= 0.00390625f;
-          sv[h] = __uint_as_float(__float_as_uint(v) & 0xFFFFFFFCu);
+          for (int h = 0; h < 2; ++h) {
+            float x = sv[h];
+            if (int4_step) x *= 0.00390625f;
+            sv[h] = __uint_as_float(__float_as_uint(x) & 0xFFFFFFFCu);
+          }
+          reinterpret_cast<float4 *>(ss)[k] =
+              make_float4(sv[0], sv[1], -gemm_cfg::kBiasF * sv[0], -gemm_cfg::kBiasF * sv[1]);
         }
-        reinterpret_cast<float4 *>(ss)[j] =
-            make_float4(sv[0], sv[1], -gemm_cfg::kBiasF * sv[0], -gemm_cfg::kBiasF * sv[1]);
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&pempty[p0.idx]);
-        if (!int4_group) mbar_arrive(&pempty[p1.idx]);
+        if (two) mbar_arrive(&pempty[p1.idx]);
         mbar_arrive(&sfull[sl]);
         mbar_arrive(&ufull[u]);
       }
       pr = p1;
-      if (!int4_group) pr.next(kNP);
+      if (two) pr.next(kNP);
     }
   }
 
