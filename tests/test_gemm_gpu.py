@@ -227,6 +227,26 @@ def test_split_k_output_matches_oracle_and_unsplit(c_oracle, M, N, K, seed):
         assert err <= Y_TOL, err
 
 
+@pytest.mark.parametrize("N,S", [(8192, 2), (5120, 3), (4096, 4), (3584, 5), (3072, 6),
+                                 (2688, 7), (2304, 8)])
+def test_small_m_every_cluster_size(c_oracle, N, S):
+    """The small-M kernel splits K over a cluster of S CTAs, S = 2 .. 8 as the
+    weight tiles fill the 148 SMs, and sums the ranges' partial tiles in
+    distributed shared memory, each CTA a slice of the rows (slices of 4-row
+    quads, uneven when S does not divide 32). Y must be within tolerance of
+    the oracle, split and unsplit."""
+    M, K = 17, 2048
+    assert atom.atom_gemm_workspace_bytes(M, N, K) == S * M * N * 4
+    A, W, idx = inputs.random_case(40 + S, M, N, K, dist="t", param=4.0, outlier_factor=30.0)
+    qa, qw = quant_dev(A, idx), quant_dev(W, idx, weights=True)
+    y_split = atom.atom_w4a4_gemm(qa, qw, K).cpu().numpy()
+    y_plain = atom.atom_w4a4_gemm(qa, qw, K, split=False).cpu().numpy()
+    ra, rw = c_oracle.quantize(A, idx), c_oracle.quantize(W, idx)
+    Y64 = c_oracle.gemm(*ra, *rw, K)
+    for y in (y_split, y_plain):
+        assert y_rel_err(y, Y64) <= Y_TOL
+
+
 def test_split_k_is_deterministic_and_ignores_a_short_workspace():
     M, N, K = 64, 4096, 4096
     A, W, idx = inputs.random_case(25, M, N, K)

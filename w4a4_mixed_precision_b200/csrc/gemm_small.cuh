@@ -217,24 +217,26 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
   uint8_t *sring = smem + kSOff;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kNP; ++s) {
-      mbar_init(&pfull[s], 33);  // 32 lanes' sa-copy arrivals + the expect_tx arrival
-      mbar_init(&pempty[s], kUnpackWarps);
+  // barriers: lane i of warp 0 initialises entry i of each ring's pair
+  static_assert(kNP <= 32 && kUS <= 32 && kSS <= 32 && kBS <= 32, "barrier init");
+  if (warp == 0) {
+    if (lane < kNP) {
+      mbar_init(&pfull[lane], 33);  // 32 lanes' sa-copy arrivals + the expect_tx arrival
+      mbar_init(&pempty[lane], kUnpackWarps);
     }
-    for (int s = 0; s < kUS; ++s) {
-      mbar_init(&ufull[s], kUnpackWarps);
-      mbar_init(&uempty[s], 1);
+    if (lane < kUS) {
+      mbar_init(&ufull[lane], kUnpackWarps);
+      mbar_init(&uempty[lane], 1);
     }
-    for (int s = 0; s < kSS; ++s) {
-      mbar_init(&sfull[s], kUnpackWarps);
-      mbar_init(&sempty[s], kDrainWarps);
+    if (lane < kSS) {
+      mbar_init(&sfull[lane], kUnpackWarps);
+      mbar_init(&sempty[lane], kDrainWarps);
     }
-    for (int i = 0; i < kBS; ++i) {
-      mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], kDrainWarps);
+    if (lane < kBS) {
+      mbar_init(&tfull[lane], 1);
+      mbar_init(&tempty[lane], kDrainWarps);
     }
-    *abort_flag = 0;
+    if (lane == 0) *abort_flag = 0;
     fence_mbar_init();
   }
   // the bias tiles: element (row, k = 0) = 6144 (A) or 2048 (B), all else 0
@@ -582,34 +584,41 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
     const int S = p.splits;
     const int rank = static_cast<int>(cluster_cta_rank());
     const int n0 = (static_cast<int>(blockIdx.x) / S) * BW;
-    const int lo = rank * BW / S, nr = (rank + 1) * BW / S - lo;
+    // this CTA's slice: weight-row quads [qlo, qlo + nq) of the tile's BW/4
+    const int qlo = rank * (BW / 4) / S, nq = (rank + 1) * (BW / 4) / S - qlo;
+    const int lo = 4 * qlo;
     const float *part = reinterpret_cast<const float *>(uring);
-    constexpr int kE = 4;                 // elements per thread in flight
-    const int total = p.M * nr;
-    for (int e0 = threadIdx.x; e0 < total; e0 += kE * threads_for(NT)) {
-      float v[kE][kMaxSplits];
+    // one thread per token and quad of weight rows: a 16-byte load from each
+    // K range's tile (all issued before the first add), the ranges added in
+    // order, one 8-byte store of 4 fp16 values (rows and N are multiples of 4)
+    const int total = p.M * nq;
+    for (int e = threadIdx.x; e < total; e += threads_for(NT)) {
+      const int m = e / nq, row = lo + 4 * (e - m * nq);
+      const float *src = part + m * BW + row;
+      float4 v[kMaxSplits];
 #pragma unroll
-      for (int u = 0; u < kE; ++u) {
-        const int e = e0 + u * threads_for(NT);
-        if (e < total) {
-          const int m = e / nr, row = lo + (e - m * nr);
-          const float *src = part + m * BW + row;
+      for (int r = 0; r < kMaxSplits; ++r)
+        if (r < S) v[r] = ld_shared_cluster_v4(cluster_map(src, r));
+      float4 a = v[0];
 #pragma unroll
-          for (int r = 0; r < kMaxSplits; ++r)
-            if (r < S) v[u][r] = ld_shared_cluster_f32(cluster_map(src, r));
+      for (int r = 1; r < kMaxSplits; ++r) {
+        if (r < S) {
+          a.x += v[r].x;
+          a.y += v[r].y;
+          a.z += v[r].z;
+          a.w += v[r].w;
         }
       }
+      __half *dst = p.y + static_cast<int64_t>(m) * p.N + n0 + row;
+      const __half2 h01 = __floats2half2_rn(a.x, a.y), h23 = __floats2half2_rn(a.z, a.w);
+      if (n0 + row + 3 < p.N) {
+        *reinterpret_cast<uint2 *>(dst) = make_uint2(*reinterpret_cast<const uint32_t *>(&h01),
+                                                     *reinterpret_cast<const uint32_t *>(&h23));
+      } else {
+        const float f[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-      for (int u = 0; u < kE; ++u) {
-        const int e = e0 + u * threads_for(NT);
-        if (e < total) {
-          const int m = e / nr, row = lo + (e - m * nr);
-          float acc = v[u][0];
-#pragma unroll
-          for (int r = 1; r < kMaxSplits; ++r)
-            if (r < S) acc += v[u][r];
-          if (n0 + row < p.N) p.y[static_cast<int64_t>(m) * p.N + n0 + row] = __float2half_rn(acc);
-        }
+        for (int c = 0; c < 4; ++c)
+          if (n0 + row + c < p.N) dst[c] = __float2half_rn(f[c]);
       }
     }
     cluster_sync();   // no CTA leaves while a peer may still read its tile
