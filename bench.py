@@ -297,6 +297,17 @@ def per_config_legs(configs, dev, stream, n_calls, int8_peak, int8_probe, hbm_gb
             return lambda: atom.atom_reorder_quant(As[i], idx, out=qouts[i], stream=st)
         q_ms = _time_cycle([quant_fn(i, stream) for i in range(n_qsets)], n_calls, stream)
         q_ms_graph = _time_graph([quant_fn(i, gs) for i in range(n_qsets)], n_calls, gs)
+
+        # one layer's online step: quantize A, then the GEMM on those codes
+        def step_fn(i, st):
+            qo, j = qouts[i % n_qsets], i % n_sets
+
+            def f():
+                atom.atom_reorder_quant(As[i % n_qsets], idx, out=qo, stream=st)
+                atom.atom_w4a4_gemm(qo, qws[j], w.K, y=ys[j], stream=st, workspace=wss[j])
+            return f
+        st_ms_graph = _time_graph([step_fn(i, gs) for i in range(max(n_sets, n_qsets))],
+                                  n_calls, gs)
         del As, qouts, qas, ys, wss
         n_csets = _copies_for(2.0 * (w.M + w.N) * w.K + 2.0 * w.M * w.N)
         Ws = [W16] + [W16.clone() for _ in range(n_csets - 1)]
@@ -323,6 +334,7 @@ def per_config_legs(configs, dev, stream, n_calls, int8_peak, int8_probe, hbm_gb
             "gemm_splits_workspace_bytes": atom.atom_gemm_workspace_bytes(w.M, w.N, w.K),
             "quant_us": round(q_ms * 1e3, 2),
             "quant_us_graph": round(q_ms_graph * 1e3, 2),
+            "step_us_graph": round(st_ms_graph * 1e3, 2),
             "quant_bytes": quant_bytes,
             "quant_gbs": round(quant_bytes / (q_ms * 1e-3) / 1e9, 1),
             "quant_frac_hbm": round(quant_bytes / (q_ms * 1e-3) / 1e9 / hbm_gbs, 4),
@@ -333,7 +345,8 @@ def per_config_legs(configs, dev, stream, n_calls, int8_peak, int8_probe, hbm_gb
             "calls": n_calls,
             "timing": "*_us: CUDA events around `calls` calls issued back to back from Python "
                       "(host launch cost included); *_us_graph: the same calls captured in one "
-                      "CUDA graph and replayed (device time per call)",
+                      "CUDA graph and replayed (device time per call); step_us_graph: quantize "
+                      "then GEMM, one layer's online step, per step in a graph",
             "l2": f"GEMM rotates {n_sets} input sets, quantizer {n_qsets}, cuBLAS {n_csets} "
                   f"weight copies (each rotation more than twice the 126 MB L2, or 16 sets)",
             "bound": "hbm" if c == 1 else "tensor",

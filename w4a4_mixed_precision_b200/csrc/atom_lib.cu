@@ -119,11 +119,23 @@ atom_status_t launch_quant(const void *x, int64_t rows, int64_t K, int64_t ld,
   // quantizer calls of this device are in flight at once.
   const int slot = static_cast<int>(dev->quant_calls.fetch_add(1, std::memory_order_relaxed) %
                                     static_cast<uint32_t>(atomk::kQuantSlots));
-  atomk::reorder_quant_kernel<<<grid, atomk::kQuantThreads, L.total,
-                                reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __half *>(x), rows, static_cast<int>(K), ld, idx, q4, q8, scales,
-      static_cast<int>(stages), static_cast<int>(crews), a8 ? 1 : 0, slot);
-  return cudaGetLastError() == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
+  // programmatic dependent launch: the kernel's set-up may overlap the end of
+  // the previous kernel in the stream (it waits for that kernel before it
+  // touches its inputs or outputs)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(atomk::kQuantThreads, 1, 1);
+  cfg.dynamicSmemBytes = L.total;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  const cudaError_t err = cudaLaunchKernelEx(
+      &cfg, atomk::reorder_quant_kernel, static_cast<const __half *>(x), rows, static_cast<int>(K),
+      ld, idx, q4, q8, scales, static_cast<int>(stages), static_cast<int>(crews), a8 ? 1 : 0, slot);
+  return err == cudaSuccess ? ATOM_OK : ATOM_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------- GEMM
@@ -321,13 +333,17 @@ atom_status_t launch_gemm_small(DeviceState *dev, const uint8_t *qa4, const int8
   cfg.blockDim = dim3(threads_for(nt), 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = static_cast<unsigned>(splits);
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
+  // the K ranges of a tile as one cluster; programmatic dependent launch as
+  // for the quantizer
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = static_cast<unsigned>(splits);
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 2;
   cudaError_t err;
   if (partials != nullptr) {
     if (M <= 16)

@@ -217,6 +217,7 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
   uint8_t *sring = smem + kSOff;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  launch_dependents();   // the next kernel may start its set-up beside this one
   // barriers: lane i of warp 0 initialises entry i of each ring's pair
   static_assert(kNP <= 32 && kUS <= 32 && kSS <= 32 && kBS <= 32, "barrier init");
   if (warp == 0) {
@@ -247,6 +248,9 @@ w4a4_gemm_small_kernel(const __grid_constant__ SmallMaps maps, const SmallParams
   }
   fence_proxy_async_smem();
   __syncthreads();
+  // the set-up above touches no input or output: from here on, the kernel
+  // before this one in the stream has completed
+  grid_dependency_wait();
   const int64_t iters = small_iterations(p);   // groups (producer)
   const int64_t steps = small_steps(p);        // steps (unpack, MMA, drain)
 

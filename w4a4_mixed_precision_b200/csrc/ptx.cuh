@@ -26,6 +26,23 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ dependent launch
+
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization may start while the kernel before it in the stream is still
+// running. grid_dependency_wait() returns once that kernel has completed and
+// its writes are visible (at once if it was not launched that way, or there is
+// no such kernel); nothing may read this kernel's inputs or write its outputs
+// before it. launch_dependents() lets the next such kernel start its own
+// set-up as soon as every CTA of this one has issued it (or exited).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {

@@ -143,8 +143,7 @@ reorder_quant_cta(uint8_t *smem, const __half *__restrict__ x, int64_t rows, int
   const int crew = warp / (kQuantWarps + 1), cw = warp % (kQuantWarps + 1);
   const int G = K / 128, Gd = G - 1, Kd = K - 128;
   const int64_t q4_row = Kd / 2;
-  // the outlier list is read once, as early as possible
-  const int oc = tid < 128 ? __ldg(outlier_idx + tid) : 0;
+  launch_dependents();   // the next kernel may start its set-up beside this one
 
   if (tid == 0) {
     for (int s = 0; s < stages_n * crews_n; ++s) {
@@ -161,6 +160,10 @@ reorder_quant_cta(uint8_t *smem, const __half *__restrict__ x, int64_t rows, int
     divtab[f] = make_float2(__fdiv_rn(m, 7.f), __fdiv_rn(7.f, m));
   }
   __syncthreads();
+  // the set-up above touches no input or output: from here on, the kernel
+  // before this one in the stream has completed
+  grid_dependency_wait();
+  const int oc = tid < 128 ? __ldg(outlier_idx + tid) : 0;
 
   // This crew's ring: stages_n slots with their barriers and row tags.
   uint64_t *cfull = full + crew * stages_n;
