@@ -25,7 +25,12 @@
  *    2i (low nibble) and 2i+1 (high nibble) as 4-bit two's complement.
  *    q8 layout: int8 [rows][128]. scales: float32 [G][rows] (group-major).
  *  - Every pointer is device memory owned by the caller; the library never
- *    allocates, frees or synchronises. Work is enqueued on `stream`.
+ *    allocates, frees or synchronises. Work is enqueued on `stream`, in stream
+ *    order. The quantizers and the GEMM for M <= 64 are launched with
+ *    programmatic stream serialization: their set-up may run while the
+ *    previous kernel in the stream finishes. They read no input and write no
+ *    output before that kernel has completed, so the ordering a caller sees is
+ *    plain stream order.
  *  - Errors a host check can see (null pointers, sizes, alignment, unsupported
  *    parameters) are returned before anything is launched. Errors only the
  *    device can see (a repeated or out-of-range outlier index, a bounded wait
