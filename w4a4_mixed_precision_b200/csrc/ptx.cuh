@@ -201,18 +201,6 @@ __device__ __forceinline__ void cp_async_4(uint32_t dst_smem, const void *src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst_smem), "l"(src) : "memory");
 }
 
-// Closes this thread's current group of cp.async copies.
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// Waits until at most N of this thread's committed cp.async groups are still
-// in flight (the older ones have landed and are visible to this thread).
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // Arrives on `bar` (without raising its expected count: the barrier's count
 // must include this arrival) once every cp.async this thread issued so far
 // has completed.
@@ -323,14 +311,6 @@ __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
-// Same with 8 consecutive columns.
-__device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                 "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
-}
-
 __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[8]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;"
                : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
@@ -381,12 +361,6 @@ __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t cluster_addr) {
   return v;
 }
 
-// Arrive on an mbarrier anywhere in the cluster (release at cluster scope).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
 // Arrive on an mbarrier anywhere in the cluster with no memory ordering. A
 // cluster-scope release arrive costs ~0.5 us more on B200; use this where
 // the signalled event carries no memory writes (e.g. "TMEM columns read",
@@ -405,62 +379,9 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_addr,
-                                                              uint32_t bytes) {
-  asm volatile(
-      "mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
-          cluster_addr),
-      "r"(bytes)
-      : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __noinline__ bool mbar_wait_cluster_slow(uint64_t *bar, uint32_t parity,
-                                                    const volatile int *abort_flag) {
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((i & 63u) == 0) {
-      if (abort_flag != nullptr && *abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) return false;
-    }
-  }
-}
-
-// Bounded wait with cluster-scope acquire, for a barrier whose arrivals
-// release writes that this thread's own generic loads must see.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
-                                                  const volatile int *abort_flag) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  return mbar_wait_cluster_slow(bar, parity, abort_flag);
-}
-
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
-}
-
-// 2-D tensor copy into this CTA's shared memory whose completion is signalled
-// on an mbarrier of the CTA pair's leader (cluster address), for operands of
-// a 2-SM MMA. No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, int32_t x,
-                                                 int32_t y, uint32_t leader_bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(leader_bar)
-      : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05, CTA pairs
@@ -546,41 +467,6 @@ __device__ __forceinline__ void tc_commit_pair_multicast(uint64_t *bar, uint16_t
       : "memory");
 }
 
-// 16 TMEM lanes x 256 bits, two 8-column blocks: thread t receives
-//   r[0], r[1]: lane (t/4),     columns 2*(t%4), 2*(t%4)+1
-//   r[2], r[3]: lane (t/4 + 8), same columns
-//   r[4..7]   : the same for the next 8 columns.
-__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                 "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
-}
-
-// 16 TMEM lanes x 256 bits, four 8-column blocks: block k of the load lands in
-// r[4k..4k+3] with the same per-thread layout as the .x2 form above.
-__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-
-// Writes `v` to 4 consecutive columns of this thread's TMEM lane. (The wider
-// forms take one register per column, which the compiler materialises as
-// copies of `v`: 16 of them overflow the drain's register budget.)
-__device__ __forceinline__ void tmem_st_x4_fill(uint32_t taddr, uint32_t v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %1, %1, %1};" ::"r"(taddr), "r"(v)
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
 // ------------------------------------------------------------------ named barriers
 
 // Barrier among `nthreads` threads (a multiple of 32) on hardware barrier `id`.
@@ -588,36 +474,7 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Same, returning the OR of `pred` over the participating threads (every
-// participant gets the same answer, so it can drive a common control decision).
-__device__ __forceinline__ bool named_bar_any(uint32_t id, uint32_t nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-
 // ------------------------------------------------------------------ packed fp32 pairs
-
-__device__ __forceinline__ float2 f2_add(float2 a, float2 b) {
-  float2 c;
-  asm("add.rn.f32x2 %0, %1, %2;"
-      : "=l"(reinterpret_cast<uint64_t &>(c))
-      : "l"(reinterpret_cast<const uint64_t &>(a)), "l"(reinterpret_cast<const uint64_t &>(b)));
-  return c;
-}
-
-__device__ __forceinline__ float2 f2_mul(float2 a, float2 b) {
-  float2 c;
-  asm("mul.rn.f32x2 %0, %1, %2;"
-      : "=l"(reinterpret_cast<uint64_t &>(c))
-      : "l"(reinterpret_cast<const uint64_t &>(a)), "l"(reinterpret_cast<const uint64_t &>(b)));
-  return c;
-}
 
 __device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
   float2 d;
@@ -632,17 +489,6 @@ __device__ __forceinline__ float2 f2_fma(float2 a, float2 b, float2 c) {
 __device__ __forceinline__ uint32_t pack_half2_rn(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// Exact int32 -> fp32 conversion for |p| < 2^22, as bits: keeps the low 23
-// bits of p with bit 22 flipped (that is p + 2^22 mod 2^23) under the exponent
-// of 2^23, so the float equals 1.5*2^23 + p. One LOP3 (select by the mask
-// 0x007FFFFF between p ^ 0x4B400000 and 0x4B400000), which runs on the
-// integer ALU pipe and leaves the FMA pipe to the scale arithmetic.
-__device__ __forceinline__ uint32_t biased_float_bits(uint32_t p) {
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(r) : "r"(p), "r"(0x007FFFFFu), "r"(0x4B400000u));
   return r;
 }
 
