@@ -21,6 +21,8 @@
 
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace atomk {
 
 constexpr int kKvThreads = 256;
@@ -87,15 +89,16 @@ kv_dequant_kernel(const uint8_t *__restrict__ q4, const float *__restrict__ scal
     uint32_t o[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      // byte j: element 2j in the low nibble, 2j+1 in the high nibble; shift each
-      // nibble to the top of a 32-bit word and back to sign-extend it
-      const uint32_t byte = (w[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-      const int32_t lo = static_cast<int32_t>(byte << 28) >> 28;
-      const int32_t hi = static_cast<int32_t>(byte << 24) >> 28;
-      const float f0 = __fmul_rn(static_cast<float>(lo), s);
-      const float f1 = __fmul_rn(static_cast<float>(hi), s);
-      o[j] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(f0))) |
-             (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(f1))) << 16);
+      // byte j: element 2j in the low nibble, 2j+1 in the high nibble. A
+      // nibble n is the code q = (n ^ 8) - 8; fp32(q) is made without a
+      // conversion instruction, as the float with bits 0x4B400000 | (n ^ 8)
+      // (= 1.5*2^23 + (n ^ 8)) minus 1.5*2^23 + 8, both steps exact. The pair
+      // of products goes to fp16 in one packed round-to-nearest conversion.
+      const uint32_t byte = w[j >> 2] >> (8 * (j & 3));
+      const float q0 = __fsub_rn(__uint_as_float(0x4B400000u | ((byte & 0xFu) ^ 8u)), 12582920.f);
+      const float q1 =
+          __fsub_rn(__uint_as_float(0x4B400000u | (((byte >> 4) & 0xFu) ^ 8u)), 12582920.f);
+      o[j] = pack_half2_rn(__fmul_rn(q0, s), __fmul_rn(q1, s));
     }
     uint4 *dst = reinterpret_cast<uint4 *>(out + g * 128 + sub * 16);
     dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
