@@ -469,6 +469,15 @@ def main():
     elapsed_ms = t_start.elapsed_time(t_end)
     quant_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n_steps)]
     gemm_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(n_steps)]
+
+    # the quantizer alone: 20 launches back to back on two alternating inputs
+    # (each larger than L2), with no GEMM in between whose Y write-backs share
+    # the quantizer's HBM time
+    A2, qa2 = A.clone(), atom.empty_quantized(w.M, w.K, dev)
+    quant_alone_ms = _time_cycle(
+        [lambda: atom.atom_reorder_quant(A, idx, out=qa, stream=stream),
+         lambda: atom.atom_reorder_quant(A2, idx, out=qa2, stream=stream)], 20, stream)
+    del A2, qa2
     elapsed_ms = parallel.max_over_ranks(elapsed_ms, dev)   # the slowest rank's time
 
     # -------- end-to-end through the public API with host buffers
@@ -783,6 +792,12 @@ def main():
             "traffic": _profiled_traffic("reorder_quant_kernel") if profiled_shape else None,
             "algorithmic_bytes": quant_bytes,
             "peak_source": f"{peak_kind} HBM copy",
+            "alone": {
+                "achieved": round(quant_bytes / (quant_alone_ms * 1e-3) / 1e9, 1),
+                "frac": round(quant_bytes / (quant_alone_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                "ms": round(quant_alone_ms, 4),
+                "how": "20 launches back to back on two alternating copies of A, no GEMM between",
+            },
         },
         "clocks": clocks.summary(),
         "gpu_launches": 2 * n_steps,
