@@ -35,10 +35,16 @@
 //    group costs each drain warp one 16-column TMEM load; an fp16 MMA of
 //    constant tiles starts each group's accumulator at the conversion bias (as
 //    in gemm.cuh), so the drain writes nothing back to TMEM;
-//  * four accumulators, so the MMA can run up to three groups ahead of the drain;
-//  * the split-K reduction issues all of an element's distributed-shared-memory
-//    loads before it adds them (in K-range order), four elements per thread at
-//    a time.
+//  * the unpack, MMA and drain roles advance two INT4 groups per step, so each
+//    crosses one barrier hand-off per two groups (a hand-off costs a few
+//    hundred ns on this part, about as much as a group's work);
+//  * four accumulators, two steps of two;
+//  * the split-K reduction gives each CTA a slice of 4-row quads: one 16-byte
+//    distributed-shared-memory load per K range, all issued before the first
+//    add (in K-range order), one 8-byte store of 4 fp16 values;
+//  * launched with programmatic stream serialization: the set-up runs while
+//    the previous kernel in the stream finishes, and nothing reads an input
+//    or writes an output before griddepcontrol.wait.
 //
 // Roles: warp 0 producer (lane 0 issues the tensor copies, all lanes the sa
 // copies); warp 1 allocates TMEM, its lane 0 issues the MMAs; warps 2..7 unpack

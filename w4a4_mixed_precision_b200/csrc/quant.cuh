@@ -24,6 +24,10 @@
 //    turn, one per call; the last CTA of a launch to finish puts its slot back
 //    to zero, so the slot is ready for its next call, or for the next replay
 //    of a captured launch;
+//  * launched with programmatic stream serialization: the barrier set-up and
+//    the scale table are built while the previous kernel in the stream
+//    finishes; the outlier list, the rows and the outputs are touched only
+//    after griddepcontrol.wait;
 //  * at start-up each CTA (once per SM, shared by its crews) turns the outlier
 //    list into a gather table in shared
 //    memory (uint16 [K]): for every group and lane, the byte offsets inside a
